@@ -1,0 +1,234 @@
+/*
+ * pgd.h -- C ABI of libpgd.so: paged GQA decode attention on B200 (sm_100a).
+ *
+ * Decode-phase attention over a paged KV cache: each running sequence has one
+ * query token, which attends over that sequence's whole cached K/V history.
+ * The history is read block by block through a block table; the query heads
+ * of a GQA group share one KV head; every sequence in the batch has its own
+ * context length; the work is split along the KV length and the splits are
+ * merged by log-sum-exp.
+ *
+ * Sources (page title and section):
+ *   "attention kernels" (froggydisk, LLM serving / decoding):
+ *     section "standard attention"      -- S = Q K^T, P = softmax(S), O = P V
+ *     section "FlashAttention"          -- online softmax over K blocks is exact
+ *     section "prefill and decode attention" -- decode reads each KV head once
+ *        for all query heads of its group; the work is split along the KV
+ *        length and the splits are merged like the online softmax
+ *     section "paged KV and kernels"    -- block table; variable-length batch
+ *        in one launch; FP8 KV read directly
+ *   "Optimization 1: batching and attention" (beengineer500):
+ *     section 2.4 -- num_attention_heads / num_key_value_heads; 32/8 = 4 heads
+ *        share one KV head
+ *     section 3.4 -- PagedAttention: fixed-size blocks, block table from
+ *        logical to physical block, blocks need not be contiguous
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are caller-owned device memory; nothing is freed or
+ *     kept past the call except the library's own workspace (see below).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call only enqueues work on `stream`; none synchronises
+ *     with the host, so results are ready once the stream has reached them.
+ *   - Host-side argument checks run before any launch and return a status;
+ *     on error nothing is enqueued.
+ *   - Faults the device detects (a block id outside [0, num_blocks), a
+ *     context length outside [0, max_blocks_per_seq * block_size], a slot
+ *     outside the pool, a pipeline wait that ran out of time) never trap:
+ *     the kernel records a flag, keeps every access in bounds and returns;
+ *     pgd_get_device_error() reports and clears the flags.  Outputs of a call
+ *     that raised a flag are undefined.
+ *
+ * KV cache layout ("HND"): k_cache and v_cache are
+ *     [num_blocks][num_kv_heads][block_size][head_dim]
+ * elements of the cache type (bf16, or FP8 E4M3 bytes), so one (block, KV
+ * head) tile of block_size x head_dim is contiguous.  Token t of sequence s
+ * lives in physical block block_table[s][t / block_size] at row
+ * t % block_size.  Query head i reads KV head i / g, g = num_q_heads /
+ * num_kv_heads.
+ */
+#ifndef PGD_H_
+#define PGD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PGD_OK = 0,
+    PGD_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer   */
+    PGD_ERR_UNSUPPORTED = 2,   /* shape outside the compiled variants          */
+    PGD_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed            */
+    PGD_ERR_DEVICE_BOUNDS = 4, /* device flagged an out-of-range index         */
+    PGD_ERR_TIMEOUT = 5,       /* device flagged a pipeline wait that timed out */
+    PGD_ERR_WORKSPACE = 6      /* caller workspace too small                   */
+} pgd_status;
+
+typedef enum {
+    PGD_KV_BF16 = 0,           /* bf16 K/V, 2 bytes per element                 */
+    PGD_KV_FP8_E4M3 = 1        /* FP8 E4M3 K/V bytes times a per-KV-head scale  */
+} pgd_kv_dtype;
+
+/* Human-readable name of a status code (static string). */
+const char *pgd_status_string(pgd_status status);
+
+/* Library version, "major.minor.patch" (static string). */
+const char *pgd_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* KV append                                                                */
+/* ------------------------------------------------------------------------ */
+/*
+ * pgd_kv_append -- write the K and V rows of new tokens into their cache
+ * slots ("batching and attention" 3.4: a token's KV lives in a slot of a
+ * fixed-size physical block).
+ *
+ *   k_new, v_new   device, [num_tokens][num_kv_heads][head_dim] elements of
+ *                  the cache type (bf16, or E4M3 bytes), 16-byte aligned.
+ *   slot_mapping   device int64 [num_tokens]; token t goes to physical block
+ *                  slot / block_size, row slot % block_size.  A slot < 0 is a
+ *                  padding token and is skipped; a slot >= num_blocks *
+ *                  block_size is skipped and flags PGD_ERR_DEVICE_BOUNDS.
+ *   k_cache, v_cache  device, HND layout above, 16-byte aligned; rows that no
+ *                  token maps to are left untouched.
+ *   num_tokens >= 0 (0 enqueues nothing); head_dim in {128, 256};
+ *   block_size in {16, 32, 64}; num_kv_heads >= 1.
+ * The copy is bit-exact.  Two tokens mapped to the same slot race (the
+ * result is one of them).
+ */
+pgd_status pgd_kv_append(const void *k_new, const void *v_new,
+                         const int64_t *slot_mapping, int32_t num_tokens,
+                         void *k_cache, void *v_cache,
+                         int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                         int32_t num_blocks, pgd_kv_dtype kv_dtype, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Paged decode attention                                                   */
+/* ------------------------------------------------------------------------ */
+/*
+ * pgd_decode_workspace_bytes -- bytes of device workspace that
+ * pgd_paged_decode_attention needs on the current device with an automatic
+ * grid (the split partial outputs and their log-sum-exps; no zeroing
+ * needed).  num_seqs is accepted for interface stability; the size depends
+ * on the group size, head_dim and the device's SM count.  Returns 0 for
+ * invalid sizes.
+ */
+size_t pgd_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
+                                  int32_t num_kv_heads, int32_t head_dim);
+
+/*
+ * pgd_paged_decode_attention -- one decode step of attention for a batch.
+ *
+ * For sequence s and query head i (KV head h = i / g), with n = context_lens[s]:
+ *   x_t   = scale * sum_d q[s][i][d] * K_t[d]            t = 0..n-1
+ *   out   = sum_t exp(x_t - M) V_t / sum_t exp(x_t - M),  M = max_t x_t
+ *   lse   = M + ln sum_t exp(x_t - M)
+ * where K_t, V_t are row t % block_size of physical block
+ * block_table[s][t / block_size], KV head h ("attention kernels", sections
+ * "standard attention" and "paged KV and kernels").  For FP8 E4M3 caches
+ * K_t = e4m3(byte) * k_scale[h] and V_t = e4m3(byte) * v_scale[h].
+ * n = 0 gives out = 0 and lse = -inf.
+ *
+ * The work of the whole batch is divided evenly over a grid sized to the
+ * device: each CTA streams an equal share of the (sequence, KV head, block)
+ * tiles through a TMA shared-memory pipeline, reads each K/V tile once for
+ * all g query heads of its group, and keeps an online softmax; a sequence
+ * whose tiles fall into several CTAs is merged by log-sum-exp by the CTA that
+ * finishes its last share ("prefill and decode attention").  The result does
+ * not depend on where the blocks sit in the pool.
+ *
+ *   q             device bf16 [num_seqs][num_q_heads][head_dim], 4-byte aligned
+ *   k_cache, v_cache  device, HND layout, 16-byte aligned, num_blocks blocks
+ *   block_table   device int32 [num_seqs][max_blocks_per_seq]; entries past
+ *                 ceil(context_lens[s] / block_size) are never read
+ *   context_lens  device int32 [num_seqs], each in [0, max_blocks_per_seq *
+ *                 block_size]
+ *   max_context_len  host hint >= every context length (0 = unknown); only
+ *                 used to size the grid for small batches
+ *   num_q_heads % num_kv_heads == 0, g = num_q_heads / num_kv_heads in
+ *                 {1, 2, 4, 8, 16}; head_dim in {128, 256} (256 with bf16
+ *                 only); block_size in {16, 32, 64}
+ *   scale         softmax scale applied to q.k (e.g. 1/sqrt(head_dim))
+ *   kv_dtype      PGD_KV_BF16 or PGD_KV_FP8_E4M3
+ *   k_scale, v_scale  device fp32 [num_kv_heads] for FP8 (NULL for bf16)
+ *   out           device bf16 [num_seqs][num_q_heads][head_dim] (RNE from fp32)
+ *   lse_out       optional device fp32 [num_seqs][num_q_heads] (natural log),
+ *                 NULL to skip
+ *   workspace, workspace_bytes  device scratch for the split partials, at
+ *                 least pgd_decode_workspace_bytes(...) bytes (any contents);
+ *                 NULL/0 selects a library-owned buffer (grown on demand with
+ *                 cudaMalloc, kept until pgd_shutdown()).  The library also
+ *                 keeps one int32 arrival counter per (sequence, KV head) in
+ *                 its own zeroed device buffer (grown the same way).  Calls
+ *                 that share a workspace, or run on one device at the same
+ *                 time, must not overlap on the GPU.
+ *   num_ctas      0 = automatic grid (a multiple of the SM count); > 0 forces
+ *                 that many CTAs (used to test split-count invariance)
+ *   stream        cudaStream_t as void*
+ */
+pgd_status pgd_paged_decode_attention(
+    const void *q, const void *k_cache, const void *v_cache,
+    const int32_t *block_table, int32_t max_blocks_per_seq,
+    const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t num_blocks, float scale, pgd_kv_dtype kv_dtype,
+    const float *k_scale, const float *v_scale,
+    void *out, float *lse_out,
+    void *workspace, size_t workspace_bytes, int32_t num_ctas, void *stream);
+
+/*
+ * pgd_merge_partials -- log-sum-exp merge of split results ("attention
+ * kernels", section "prefill and decode attention": splits along the KV
+ * length are merged the same way the online softmax merges blocks).  For
+ * each row r:  M = max_p lse_part[p][r];  w_p = exp(lse_part[p][r] - M);
+ * out[r] = sum_p w_p o_part[p][r] / sum_p w_p;  lse[r] = M + ln sum_p w_p.
+ * Splits with lse = -inf carry no weight; a row whose splits are all -inf
+ * gives out = 0, lse = -inf.  Used to merge per-GPU splits of one sequence.
+ *
+ *   o_part    device fp32 [num_parts][rows][head_dim]
+ *   lse_part  device fp32 [num_parts][rows] (natural log)
+ *   out       device bf16 [rows][head_dim]
+ *   lse_out   optional device fp32 [rows], NULL to skip
+ *   num_parts >= 1, rows >= 0, head_dim in {128, 256}
+ */
+pgd_status pgd_merge_partials(const float *o_part, const float *lse_part,
+                              int32_t num_parts, int32_t rows, int32_t head_dim,
+                              void *out, float *lse_out, void *stream);
+
+/*
+ * pgd_get_device_error -- wait for `stream`, then read and clear the device
+ * flags raised by earlier calls on this device.  Returns PGD_OK when none
+ * was raised, PGD_ERR_DEVICE_BOUNDS or PGD_ERR_TIMEOUT otherwise (and
+ * *flags, if non-NULL, receives the raw bit set: 1 block id, 2 context
+ * length, 4 slot, 8 wait timeout).
+ */
+pgd_status pgd_get_device_error(void *stream, uint32_t *flags);
+
+/* Free library-owned workspaces (call with no work in flight). */
+pgd_status pgd_shutdown(void);
+
+/* ------------------------------------------------------------------------ */
+/* Short forms with the argument lists of the problem statement.            */
+/* ------------------------------------------------------------------------ */
+/* kv_append for bf16 caches: pgd_kv_append with PGD_KV_BF16. */
+pgd_status kv_append(const void *k_new, const void *v_new, const int64_t *slot_mapping,
+                     int32_t num_tokens, void *k_cache, void *v_cache,
+                     int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                     int32_t num_blocks, void *stream);
+
+/* paged_decode_attention for bf16 caches, no lse output, library workspace,
+ * automatic grid: pgd_paged_decode_attention with those choices. */
+pgd_status paged_decode_attention(const void *q, const void *k_cache, const void *v_cache,
+                                  const int32_t *block_table, int32_t max_blocks_per_seq,
+                                  const int32_t *context_lens, int32_t num_seqs,
+                                  int32_t num_q_heads, int32_t num_kv_heads,
+                                  int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                                  float scale, void *out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PGD_H_ */

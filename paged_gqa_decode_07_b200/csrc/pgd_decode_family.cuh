@@ -1,0 +1,69 @@
+// pgd_decode_family.cuh -- definitions of the per-variant launchers; each
+// pgd_decode_*.cu unit includes this and instantiates one family.
+#pragma once
+
+#include <atomic>
+
+#include "pgd_launch.h"
+
+namespace pgd {
+
+template <int D, int BS, int NT, bool FP8>
+static void *decode_kernel_ptr() {
+    constexpr int NS = Stages<D, FP8>::value;
+    return reinterpret_cast<void *>(&paged_decode_kernel<D, BS, NT, FP8, NS>);
+}
+
+template <int D, int BS, int NT, bool FP8>
+static cudaError_t ensure_smem_attr() {
+    constexpr int NS = Stages<D, FP8>::value;
+    using C = DecodeCfg<D, BS, NT, FP8, NS>;
+    static std::atomic<uint64_t> done_mask{0};   // one bit per device ordinal < 64
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+    if (bit && (done_mask.load() & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(decode_kernel_ptr<D, BS, NT, FP8>(),
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e == cudaSuccess && bit) done_mask.fetch_or(bit);
+    return e;
+}
+
+template <int D, int BS, int NT, bool FP8>
+cudaError_t launch_decode(const DecodeLaunchArgs &a) {
+    constexpr int NS = Stages<D, FP8>::value;
+    using C = DecodeCfg<D, BS, NT, FP8, NS>;
+    cudaError_t e = ensure_smem_attr<D, BS, NT, FP8>();
+    if (e != cudaSuccess) return e;
+    paged_decode_kernel<D, BS, NT, FP8, NS><<<a.grid, kThreads, C::SMEM, a.stream>>>(a.tmK, a.tmV, a.p);
+    return cudaGetLastError();
+}
+
+template <int D, int BS, int NT, bool FP8>
+int decode_ctas_per_sm() {
+    constexpr int NS = Stages<D, FP8>::value;
+    using C = DecodeCfg<D, BS, NT, FP8, NS>;
+    if (ensure_smem_attr<D, BS, NT, FP8>() != cudaSuccess) return 0;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel_ptr<D, BS, NT, FP8>(),
+                                                      kThreads, C::SMEM) != cudaSuccess)
+        return 0;
+    return n;
+}
+
+#define PGD_INSTANTIATE_FAMILY(D, FP8)                                          \
+    template cudaError_t launch_decode<D, 16, 1, FP8>(const DecodeLaunchArgs &); \
+    template cudaError_t launch_decode<D, 32, 1, FP8>(const DecodeLaunchArgs &); \
+    template cudaError_t launch_decode<D, 64, 1, FP8>(const DecodeLaunchArgs &); \
+    template cudaError_t launch_decode<D, 16, 2, FP8>(const DecodeLaunchArgs &); \
+    template cudaError_t launch_decode<D, 32, 2, FP8>(const DecodeLaunchArgs &); \
+    template cudaError_t launch_decode<D, 64, 2, FP8>(const DecodeLaunchArgs &); \
+    template int decode_ctas_per_sm<D, 16, 1, FP8>();                           \
+    template int decode_ctas_per_sm<D, 32, 1, FP8>();                           \
+    template int decode_ctas_per_sm<D, 64, 1, FP8>();                           \
+    template int decode_ctas_per_sm<D, 16, 2, FP8>();                           \
+    template int decode_ctas_per_sm<D, 32, 2, FP8>();                           \
+    template int decode_ctas_per_sm<D, 64, 2, FP8>();
+
+}  // namespace pgd
