@@ -179,6 +179,43 @@ pgd_status pgd_paged_decode_attention(
     void *workspace, size_t workspace_bytes, int32_t num_ctas, void *stream);
 
 /*
+ * pgd_paged_decode_attention_noalloc -- the same decode step as
+ * pgd_paged_decode_attention, for callers that must not have the library
+ * allocate device memory: a serving engine that has reserved nearly all HBM
+ * for its KV-cache pool (a cudaMalloc at decode time can fail), a host that
+ * routes and accounts every device byte through its own allocator, or a
+ * decode loop that cannot absorb the device-wide synchronisation of a
+ * cudaFree when a library buffer grows.  There is no counterpart on the
+ * pages; this is an interface choice of the library.
+ *
+ * Arguments are those of pgd_paged_decode_attention without the workspace:
+ * the caller still provides every input and output.  The split partials and
+ * the arrival counters live in one static device array of 8 MiB per device
+ * (held by every GPU that loads the library until the process exits).  The
+ * call allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ * routine.
+ *   - Limits: num_seqs * num_kv_heads <= 65536, and the split partials of the
+ *     grid must fit in the rest of the array; an automatic grid is reduced to
+ *     fit, an explicit num_ctas that does not fit is rejected.  Requests past
+ *     a limit return PGD_ERR_WORKSPACE and enqueue nothing.
+ *   - Set-up: the first call on each device (with that device current)
+ *     resolves the array's device address with cudaGetSymbolAddress; make
+ *     that first call before any stream capture.
+ *   - Every call clears the counters it uses (a cudaMemsetAsync on `stream`)
+ *     and then reuses the array, which keeps the previous call's contents.
+ *     Calls on one device that overlap on the GPU (other streams, other host
+ *     threads) share the array and race: serialise them.
+ */
+pgd_status pgd_paged_decode_attention_noalloc(
+    const void *q, const void *k_cache, const void *v_cache,
+    const int32_t *block_table, int32_t max_blocks_per_seq,
+    const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t num_blocks, float scale, pgd_kv_dtype kv_dtype,
+    const float *k_scale, const float *v_scale,
+    void *out, float *lse_out, int32_t num_ctas, void *stream);
+
+/*
  * pgd_merge_partials -- log-sum-exp merge of split results ("attention
  * kernels", section "prefill and decode attention": splits along the KV
  * length are merged the same way the online softmax merges blocks).  For

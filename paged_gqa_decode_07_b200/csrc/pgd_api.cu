@@ -412,3 +412,152 @@ pgd_status paged_decode_attention(const void *q, const void *k_cache, const void
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------
+// Decode with no device allocation by the library.
+//
+// Some callers cannot let a library call cudaMalloc: a serving engine that
+// reserves nearly all HBM for its KV-cache pool up front (a later cudaMalloc
+// can fail, or push the pool out), a host whose policy is that every device
+// byte goes through its own allocator and is accounted there, or a tight
+// decode loop that cannot afford the device-wide synchronisation a cudaFree
+// implies when a library buffer grows.  For them the scratch this kernel
+// needs (split partials and the per-(sequence, KV head) arrival counters)
+// lives in one fixed array of static device memory, below; each GPU that
+// loads the library holds it until the process exits.
+// ----------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;    // 8 MiB per device
+constexpr long long kStaticMaxUnits = 65536;               // counters: 256 KiB
+constexpr size_t kStaticCounterBytes = sizeof(int32_t) * kStaticMaxUnits;
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+struct StaticScratch {
+    bool ready = false;
+    unsigned char *ptr = nullptr;   // device address of g_static_scratch
+};
+StaticScratch g_static[kMaxDevices];
+
+// Resolve the device address of the static array for the current device.
+// `g_static_scratch` in host code is only a stand-in symbol, so the address
+// is looked up once per device (with that device current) and cached.
+pgd_status static_scratch(unsigned char **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PGD_ERR_CUDA;
+    StaticScratch &s = g_static[dev];
+    if (!s.ready) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!s.ready) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return PGD_ERR_CUDA;
+            s.ptr = static_cast<unsigned char *>(p);
+            s.ready = true;
+        }
+    }
+    *out = s.ptr;
+    return PGD_OK;
+}
+
+}  // namespace
+
+extern "C" pgd_status pgd_paged_decode_attention_noalloc(
+    const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+    int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
+    int32_t max_context_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t num_blocks, float scale, pgd_kv_dtype kv_dtype,
+    const float *k_scale, const float *v_scale, void *out, float *lse_out, int32_t num_ctas,
+    void *stream) {
+    // same host-side checks as pgd_paged_decode_attention
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
+        max_blocks_per_seq <= 0 || max_context_len < 0 || num_ctas < 0)
+        return PGD_ERR_INVALID_ARG;
+    if (num_q_heads % num_kv_heads) return PGD_ERR_INVALID_ARG;
+    if (kv_dtype != PGD_KV_BF16 && kv_dtype != PGD_KV_FP8_E4M3) return PGD_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PGD_ERR_INVALID_ARG;
+    const int g = num_q_heads / num_kv_heads;
+    const bool fp8 = kv_dtype == PGD_KV_FP8_E4M3;
+    if (!supported_group(g) || !supported_block(block_size)) return PGD_ERR_UNSUPPORTED;
+    if (head_dim != 128 && head_dim != 256) return PGD_ERR_UNSUPPORTED;
+    if (fp8 && head_dim != 128) return PGD_ERR_UNSUPPORTED;
+    if (static_cast<long long>(num_blocks) * num_kv_heads >= INT_MAX ||
+        static_cast<long long>(max_blocks_per_seq) * block_size >= INT_MAX)
+        return PGD_ERR_UNSUPPORTED;
+    // the counters have a fixed capacity in the static array
+    const long long units = static_cast<long long>(num_seqs) * num_kv_heads;
+    if (units > kStaticMaxUnits) return PGD_ERR_WORKSPACE;
+    if (num_seqs == 0) return PGD_OK;
+    if (!q || !k_cache || !v_cache || !block_table || !context_lens || !out)
+        return PGD_ERR_INVALID_ARG;
+    if (fp8 && (!k_scale || !v_scale)) return PGD_ERR_INVALID_ARG;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 4) || !aligned(out, 2) ||
+        !aligned(block_table, 4) || !aligned(context_lens, 4) || (lse_out && !aligned(lse_out, 4)))
+        return PGD_ERR_INVALID_ARG;
+
+    DeviceState *d = nullptr;
+    pgd_status st = device_state(&d);
+    if (st != PGD_OK) return st;
+    unsigned char *scratch = nullptr;
+    if ((st = static_scratch(&scratch)) != PGD_OK) return st;
+    const int nt = g > 8 ? 2 : 1;
+    Variant var;
+    if (!pick_variant(head_dim, block_size, nt, fp8, &var)) return PGD_ERR_UNSUPPORTED;
+
+    // grid: as the allocating entry point, then capped so that the split
+    // partials fit behind the counters in the static array
+    const size_t avail = kStaticScratchBytes - kStaticCounterBytes;
+    long long grid = num_ctas;
+    if (grid == 0) {
+        const int occ = var.occ();
+        if (occ <= 0) return PGD_ERR_CUDA;
+        grid = static_cast<long long>(d->sms) * occ;
+        const long long cap_tokens = static_cast<long long>(max_blocks_per_seq) * block_size;
+        const long long max_ctx =
+            max_context_len > 0 ? std::min<long long>(max_context_len, cap_tokens) : cap_tokens;
+        const long long tiles_upper =
+            static_cast<long long>(num_seqs) * num_kv_heads * ((max_ctx + block_size - 1) / block_size);
+        const long long min_tiles = 4 * (kStageTokens / block_size);
+        grid = std::max(1LL, std::min(grid, (tiles_upper + min_tiles - 1) / min_tiles));
+        while (grid > 1 && ws_layout(g, head_dim, grid).total > avail) --grid;
+    }
+    if (grid > (1LL << 24)) return PGD_ERR_INVALID_ARG;
+    const WsLayout lay = ws_layout(g, head_dim, grid);
+    if (lay.total > avail) return PGD_ERR_WORKSPACE;   // an explicit num_ctas too large
+
+    // the counters must start at zero; the partials need no clearing
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(int32_t) * units, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+
+    DecodeLaunchArgs a;
+    std::memset(&a, 0, sizeof(a));
+    const int E = fp8 ? 1 : 2;
+    const long long rows = static_cast<long long>(num_blocks) * num_kv_heads;
+    if ((st = encode_kv_map(&a.tmK, k_cache, head_dim, E, block_size, rows)) != PGD_OK) return st;
+    if ((st = encode_kv_map(&a.tmV, v_cache, head_dim, E, block_size, rows)) != PGD_OK) return st;
+    uint8_t *parts = scratch + kStaticCounterBytes;
+    DecodeParams &p = a.p;
+    p.q = static_cast<const uint16_t *>(q);
+    p.out = static_cast<uint16_t *>(out);
+    p.lse_out = lse_out;
+    p.block_table = block_table;
+    p.context_lens = context_lens;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.counters = reinterpret_cast<int32_t *>(scratch);
+    p.lse_part = reinterpret_cast<float *>(parts + lay.lse);
+    p.o_part = reinterpret_cast<float *>(parts + lay.opart);
+    p.flags = d->flags;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_seqs = num_seqs;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.group = g;
+    p.num_blocks = num_blocks;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    a.grid = static_cast<int>(grid);
+    a.stream = s;
+    e = var.launch(a);
+    return e == cudaSuccess ? PGD_OK : cuda_fail(e);
+}
