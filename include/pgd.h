@@ -139,7 +139,7 @@ size_t pgd_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
  * finishes its last share ("prefill and decode attention").  The result does
  * not depend on where the blocks sit in the pool.
  *
- *   q             device bf16 [num_seqs][num_q_heads][head_dim], 4-byte aligned
+ *   q             device bf16 [num_seqs][num_q_heads][head_dim], 16-byte aligned
  *   k_cache, v_cache  device, HND layout, 16-byte aligned, num_blocks blocks
  *   block_table   device int32 [num_seqs][max_blocks_per_seq]; entries past
  *                 ceil(context_lens[s] / block_size) are never read
@@ -153,7 +153,8 @@ size_t pgd_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
  *   scale         softmax scale applied to q.k (e.g. 1/sqrt(head_dim))
  *   kv_dtype      PGD_KV_BF16 or PGD_KV_FP8_E4M3
  *   k_scale, v_scale  device fp32 [num_kv_heads] for FP8 (NULL for bf16)
- *   out           device bf16 [num_seqs][num_q_heads][head_dim] (RNE from fp32)
+ *   out           device bf16 [num_seqs][num_q_heads][head_dim] (RNE from fp32),
+ *                 16-byte aligned
  *   lse_out       optional device fp32 [num_seqs][num_q_heads] (natural log),
  *                 NULL to skip
  *   workspace, workspace_bytes  device scratch for the split partials, at

@@ -248,7 +248,7 @@ pgd_status pgd_paged_decode_attention(
     if (!q || !k_cache || !v_cache || !block_table || !context_lens || !out)
         return PGD_ERR_INVALID_ARG;
     if (fp8 && (!k_scale || !v_scale)) return PGD_ERR_INVALID_ARG;
-    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 4) || !aligned(out, 2) ||
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 16) || !aligned(out, 16) ||
         !aligned(block_table, 4) || !aligned(context_lens, 4) || (lse_out && !aligned(lse_out, 4)) ||
         (workspace && !aligned(workspace, 16)))
         return PGD_ERR_INVALID_ARG;
@@ -491,7 +491,7 @@ extern "C" pgd_status pgd_paged_decode_attention_noalloc(
     if (!q || !k_cache || !v_cache || !block_table || !context_lens || !out)
         return PGD_ERR_INVALID_ARG;
     if (fp8 && (!k_scale || !v_scale)) return PGD_ERR_INVALID_ARG;
-    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 4) || !aligned(out, 2) ||
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 16) || !aligned(out, 16) ||
         !aligned(block_table, 4) || !aligned(context_lens, 4) || (lse_out && !aligned(lse_out, 4)))
         return PGD_ERR_INVALID_ARG;
 

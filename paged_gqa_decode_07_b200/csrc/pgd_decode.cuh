@@ -9,20 +9,23 @@
 //
 // Work decomposition.  The batch is flattened into tiles (s, h, j): KV head h
 // of logical block j of sequence s, ordered by s, then h, then j.  The U tiles
-// are cut into gridDim.x equal contiguous ranges, one per CTA, so every CTA
-// streams the same number of KV bytes whatever the length mix ("prefill and
-// decode attention": split along the KV length so all SMs read at once).
-// Every CTA derives the cut from context_lens itself (no host round trip).
-// Inside its range a CTA walks "segments" (the part of one (s, h) unit that
-// falls in the range).  A segment that covers its whole unit writes `out`
-// directly; otherwise it writes a partial (o, lse) and the CTA that completes
-// the unit's last share merges the partials by log-sum-exp.
+// are cut into G equal contiguous ranges, one per CTA, so every CTA streams
+// the same number of KV bytes whatever the length mix ("prefill and decode
+// attention": split along the KV length so that all SMs read at once).  Every
+// CTA derives the cut from context_lens itself (no host round trip).  Inside
+// its range a CTA walks "segments" (the part of one (s, h) unit that falls in
+// the range).  A segment that covers its whole unit writes `out` directly;
+// otherwise it writes a partial (o, lse) and the CTA that completes the
+// unit's last share merges the partials by log-sum-exp.
 //
-// CTA = 4 consumer warps + 1 producer warp.  The producer walks the same
-// segments and issues one TMA tensor load per (block, KV head) tile of K and
-// of V into a ring of shared-memory stages (64 tokens each, 128-byte swizzle,
-// mbarrier completion).  Each K/V tile is fetched once and used by all g
-// query heads of the group ("prefill and decode attention": GQA reuse).
+// CTA = 4 consumer warps + 1 producer warp.  The producer is the only warp
+// that reads the inputs from global memory: it walks the segments, writes a
+// descriptor for each into a small shared-memory ring together with the
+// unit's query rows (bulk copy), loads the block-table entries 32 at a time,
+// and issues one TMA tensor load per (block, KV head) tile of K and of V into
+// a ring of 64-token stages (128-byte swizzle, mbarrier completion).  Each
+// K/V tile is fetched once and used by all g query heads of the group
+// ("prefill and decode attention": GQA reuse).
 //
 // Per stage the consumers run a small tensor-core contraction per warp
 // (mma.sync m16n8k16, fp32 accumulate) with the roles transposed so that the
@@ -42,14 +45,14 @@
 namespace pgd {
 
 struct DecodeParams {
-    const uint16_t *q;            // bf16 bits [B][Hq][D]
+    const uint16_t *q;            // bf16 bits [B][Hq][D], 16-byte aligned
     uint16_t *out;                // bf16 bits [B][Hq][D]
     float *lse_out;               // [B][Hq] natural log, may be null
     const int32_t *block_table;   // [B][max_blocks_per_seq]
     const int32_t *context_lens;  // [B]
     const float *k_scale;         // [Hkv] (FP8 only)
     const float *v_scale;
-    int32_t *counters;            // [B * Hkv], zero between calls (library-owned)
+    int32_t *counters;            // [B * Hkv], zero between calls
     float *o_part;                // [2 * grid][g][D]
     float *lse_part;              // [2 * grid][g], log2 domain
     uint32_t *flags;              // device flag word
@@ -65,6 +68,15 @@ constexpr int kStageTokens = 16 * kConsumerWarps;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kBarConsumers = 1;
 
+// Segment descriptor written by the producer, read by the consumers.
+struct SegDesc {
+    long long u;      // flattened index of the segment's first tile
+    int s, h, j0, j1, n, ctx;
+    int terminal;     // 1: no more segments for this CTA
+    float ksc, vsc;   // FP8 per-KV-head scales (1 for bf16)
+    int pad;
+};
+
 template <int D, int BS, int NT, bool FP8, int NSTAGES>
 struct DecodeCfg {
     static constexpr int E = FP8 ? 1 : 2;                // bytes per KV element
@@ -78,27 +90,33 @@ struct DecodeCfg {
     static constexpr int DW = D / kConsumerWarps;        // PV dims per warp
     static constexpr int MT = DW / 16;                   // PV m-tiles per warp
     static constexpr int KSTEPS = D / 16;                // QK k-steps
+    static constexpr int QSLOT = NP * D * 2;             // query rows of one unit
+    static constexpr int NSEG = QSLOT >= 4096 ? 2 : 4;   // descriptor ring depth
     // shared memory carve-up (offsets from a 1024-aligned base)
-    static constexpr int OFF_P = NSTAGES * STAGE;
     static constexpr int P_BYTES = kStageTokens * NP * 2;   // one weight plane
-    static constexpr int OFF_RED = OFF_P + 2 * P_BYTES;      // hi and lo planes
+    static constexpr int OFF_P = NSTAGES * STAGE;
+    static constexpr int OFF_Q = OFF_P + 2 * P_BYTES;        // hi and lo planes
+    static constexpr int OFF_SEG = OFF_Q + NSEG * QSLOT;
+    static constexpr int OFF_RED = OFF_SEG + NSEG * (int)sizeof(SegDesc);
     static constexpr int OFF_LSUM = OFF_RED + kConsumerWarps * NP * 4;
     static constexpr int OFF_BAR = OFF_LSUM + kConsumerWarps * NP * 4;
-    static constexpr int OFF_MISC = OFF_BAR + 2 * NSTAGES * 8;
+    static constexpr int NBARS = 2 * NSTAGES + 2 * NSEG;
+    static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int MISC_BYTES = 256;
     static constexpr int SMEM = OFF_MISC + MISC_BYTES + 1024;   // + alignment slack
     static_assert(ROW % 128 == 0, "rows must be whole 128-byte lines");
-    static_assert(kStageTokens % BS == 0, "stage must hold whole blocks");
+    static_assert(kStageTokens % BS == 0 && 32 % BPS == 0, "stage must hold whole blocks");
     static_assert(!FP8 || D == 128, "FP8 path is compiled for head_dim 128");
     static_assert(TILE % 1024 == 0, "tiles must keep the 1024-byte swizzle atom aligned");
+    static_assert(sizeof(SegDesc) % 16 == 0, "descriptor alignment");
 };
 
 struct Misc {                 // CTA-wide scalars in shared memory
-    long long u0, u1, total;  // tile range of this CTA, total tiles
-    long long pfx0;           // flattened index of the first tile of unit (s0, *)
+    long long pfx0;           // flattened index of the first tile of sequence s0
     int s0;
     int is_last;
     int found;
+    int pad;
     long long warp_tmp[8];
 };
 
@@ -151,13 +169,13 @@ __device__ __forceinline__ long long block_scan(long long v, long long &total, M
     return v + before;
 }
 
-// First CTA whose range contains flattened tile x (ranges are
-// [c*U/G, (c+1)*U/G)).
+// The CTA that holds flattened tile x (ranges are [c*U/G, (c+1)*U/G), all
+// non-empty since G <= U).
 __device__ __forceinline__ long long cta_of(long long x, long long U, long long G) {
     return ((x + 1) * G - 1) / U;
 }
 
-// Walk state shared by producer and consumers (same deterministic order).
+// Walk state of the producer.
 struct Cursor {
     int s, h, j, n, ctx;
     long long u;
@@ -176,9 +194,98 @@ __device__ __forceinline__ void next_unit(Cursor &c, const DecodeParams &p) {
     }
 }
 
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uint32_t bytes,
+                                              uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+
+__device__ __forceinline__ long long lds64(uint32_t a) {
+    long long v;
+    asm volatile("ld.shared.b64 %0, [%1];" : "=l"(v) : "r"(a));
+    return v;
+}
+
+// Log-sum-exp merge of one unit's split partials by the 128 consumer threads
+// ("attention kernels", "prefill and decode attention"): with lse_c in the
+// log2 domain, M = max_c lse_c, w_c = 2^(lse_c - M), out = sum w_c o_c / sum w_c.
+// Each thread owns one query head and a strided set of float4 columns; the
+// weights are formed once per head and the partial rows are read four pieces
+// at a time so that the L2 round trips overlap.
+template <int D>
+__device__ __forceinline__ void merge_unit(const DecodeParams &p, long long ua, long long U,
+                                           long long G, long long c_first, long long c_last,
+                                           long long row0, int g) {
+    constexpr int V4 = D / 4;                      // float4 columns per row
+    constexpr int MAXC = (V4 + 7) / 8;             // columns per thread when g = 16
+    const int tph = kConsumers / g;                // threads per head (g <= 16)
+    const int head = threadIdx.x / tph, sub = threadIdx.x % tph;
+    auto slot_of = [&](long long c) { return 2 * c + ((ua <= c * U / G) ? 0 : 1); };
+    // pass 1: M over the pieces
+    float M = -INFINITY;
+    long long c = c_first;
+    for (; c + 3 <= c_last; c += 4) {
+        float l[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) l[i] = __ldcg(p.lse_part + slot_of(c + i) * g + head);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) M = fmaxf(M, l[i]);
+    }
+    for (; c <= c_last; ++c) M = fmaxf(M, __ldcg(p.lse_part + slot_of(c) * g + head));
+    const float Mu = M == -INFINITY ? 0.f : M;
+    // pass 2: weighted sum of the partial rows
+    float4 acc[MAXC];
+#pragma unroll
+    for (int i = 0; i < MAXC; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float W = 0.f;
+    auto add_piece = [&](long long cc, float w) {
+        const float4 *row = reinterpret_cast<const float4 *>(p.o_part + (slot_of(cc) * g + head) * D);
+#pragma unroll
+        for (int i = 0; i < MAXC; ++i) {
+            const int col = sub + i * tph;
+            if (col < V4) {
+                const float4 v = __ldcg(row + col);
+                acc[i].x += w * v.x; acc[i].y += w * v.y; acc[i].z += w * v.z; acc[i].w += w * v.w;
+            }
+        }
+    };
+    for (c = c_first; c + 1 <= c_last; c += 2) {
+        const float w0 = ex2(__ldcg(p.lse_part + slot_of(c) * g + head) - Mu);
+        const float w1 = ex2(__ldcg(p.lse_part + slot_of(c + 1) * g + head) - Mu);
+        W += w0 + w1;
+        add_piece(c, w0);
+        add_piece(c + 1, w1);
+    }
+    if (c <= c_last) {
+        const float w0 = ex2(__ldcg(p.lse_part + slot_of(c) * g + head) - Mu);
+        W += w0;
+        add_piece(c, w0);
+    }
+    const float inv = W > 0.f ? 1.f / W : 0.f;
+#pragma unroll
+    for (int i = 0; i < MAXC; ++i) {
+        const int col = sub + i * tph;
+        if (col < V4) {
+            uint2 packed;
+            packed.x = pack_bf16x2(acc[i].x * inv, acc[i].y * inv);
+            packed.y = pack_bf16x2(acc[i].z * inv, acc[i].w * inv);
+            *reinterpret_cast<uint2 *>(p.out + (row0 + head) * D + 4 * col) = packed;
+        }
+    }
+    if (p.lse_out && sub == 0)
+        p.lse_out[row0 + head] = W > 0.f ? (M + log2f(W)) * kLn2 : -INFINITY;
+}
+
 // ------------------------------------------------------------------ kernel
 template <int D, int BS, int NT, bool FP8, int NSTAGES>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
 paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
     using C = DecodeCfg<D, BS, NT, FP8, NSTAGES>;
@@ -189,9 +296,14 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
     Misc *misc = reinterpret_cast<Misc *>(smem + C::OFF_MISC);
     float *red = reinterpret_cast<float *>(smem + C::OFF_RED);
     float *lsum = reinterpret_cast<float *>(smem + C::OFF_LSUM);
+    SegDesc *segs = reinterpret_cast<SegDesc *>(smem + C::OFF_SEG);
+    const uint32_t sSeg = sbase + C::OFF_SEG;
     const uint32_t bar_full = sbase + C::OFF_BAR;
     const uint32_t bar_empty = bar_full + NSTAGES * 8;
+    const uint32_t seg_full = bar_empty + NSTAGES * 8;
+    const uint32_t seg_empty = seg_full + C::NSEG * 8;
     const uint32_t sP = sbase + C::OFF_P;
+    const uint32_t sQ = sbase + C::OFF_Q;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int B = p.num_seqs, Hkv = p.num_kv_heads, g = p.group;
@@ -201,6 +313,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         for (int i = 0; i < NSTAGES; ++i) {
             mbar_init(bar_full + 8 * i, 1);
             mbar_init(bar_empty + 8 * i, kConsumerWarps);
+        }
+        for (int i = 0; i < C::NSEG; ++i) {
+            mbar_init(seg_full + 8 * i, 1);
+            mbar_init(seg_empty + 8 * i, kConsumerWarps);
         }
         fence_mbar_init();
         misc->found = 0;
@@ -218,17 +334,21 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
     const long long G = min((long long)gridDim.x, U);
     const long long u0 = cta < G ? cta * U / G : 0, u1 = cta < G ? (cta + 1) * U / G : 0;
 
-    // units with an empty context: out = 0, lse = -inf (spread over CTAs)
-    for (long long v = cta; v < (long long)B * Hkv; v += gridDim.x) {
+    // units with an empty context: out = 0, lse = -inf (each thread checks
+    // its own units, spread over all CTAs)
+    for (long long v = cta + (long long)gridDim.x * tid; v < (long long)B * Hkv;
+         v += (long long)gridDim.x * kThreads) {
         const int s = (int)(v / Hkv), h = (int)(v % Hkv);
         if (ctx_of<BS>(p, s) != 0) continue;
-        uint16_t *o = p.out + ((long long)s * p.num_q_heads + (long long)h * g) * D;
-        for (int e = tid; e < g * D; e += kThreads) o[e] = 0;
-        if (p.lse_out && tid < g) p.lse_out[(long long)s * p.num_q_heads + h * g + tid] = -INFINITY;
+        const long long row0 = (long long)s * p.num_q_heads + (long long)h * g;
+        uint16_t *o = p.out + row0 * D;
+        for (int e = 0; e < g * D; ++e) o[e] = 0;
+        if (p.lse_out)
+            for (int e = 0; e < g; ++e) p.lse_out[row0 + e] = -INFINITY;
     }
     if (u0 >= u1) return;   // nothing in flight, no barrier shared past this point
 
-    // locate the unit that holds tile u0
+    // locate the sequence that holds tile u0
     {
         long long base = 0;
         for (int sb = 0; sb < B; sb += kThreads) {
@@ -249,109 +369,186 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
     }
     __syncthreads();
 
-    Cursor cur;
-    cur.s = misc->s0;
-    cur.ctx = ctx_of<BS>(p, cur.s);
-    cur.n = nblk_of<BS>(cur.ctx);
-    {
-        const long long off = u0 - misc->pfx0;
-        cur.h = (int)(off / cur.n);
-        cur.j = (int)(off % cur.n);
-    }
-    cur.u = u0;
-
     if (warp == kConsumerWarps) {
-        // ================= producer: one lane issues all TMA loads ========
-        if (lane != 0) return;
-        uint32_t it = 0;
+        // ================= producer warp ====================================
+        Cursor cur;
+        cur.s = misc->s0;
+        cur.ctx = ctx_of<BS>(p, cur.s);
+        cur.n = nblk_of<BS>(cur.ctx);
+        {
+            const long long off = u0 - misc->pfx0;
+            cur.h = (int)(off / cur.n);
+            cur.j = (int)(off % cur.n);
+        }
+        cur.u = u0;
+        const uint32_t qbytes = (uint32_t)(g * D * 2);
+        uint32_t it = 0, sit = 0;
         bool ok = true;
         while (cur.u < u1 && ok) {
             const int j1 = (int)min((long long)cur.n, cur.j + (u1 - cur.u));
+            // -- descriptor and query rows of the segment
+            {
+                const uint32_t slot = sit % C::NSEG;
+                if (lane == 0 && sit >= (uint32_t)C::NSEG)
+                    ok = mbar_wait_bounded(seg_empty + 8 * slot, ((sit / C::NSEG) - 1) & 1);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                if (lane == 0) {
+                    SegDesc &d = segs[slot];
+                    d.u = cur.u;
+                    d.s = cur.s;
+                    d.h = cur.h;
+                    d.j0 = cur.j;
+                    d.j1 = j1;
+                    d.n = cur.n;
+                    d.ctx = cur.ctx;
+                    d.terminal = 0;
+                    d.ksc = FP8 ? __ldg(p.k_scale + cur.h) : 1.f;
+                    d.vsc = FP8 ? __ldg(p.v_scale + cur.h) : 1.f;
+                    const uint32_t bar = seg_full + 8 * slot;
+                    mbar_arrive_expect_tx(bar, qbytes);
+                    bulk_copy_g2s(sQ + slot * C::QSLOT,
+                                  p.q + ((long long)cur.s * p.num_q_heads + (long long)cur.h * g) * D,
+                                  qbytes, bar);
+                }
+                ++sit;
+            }
+            // -- K/V tiles, block ids fetched 32 at a time (one chunk ahead)
             const int32_t *bt = p.block_table + (long long)cur.s * p.max_blocks_per_seq;
-            for (int jj = cur.j; jj < j1 && ok; jj += C::BPS) {
-                const int nb = min(C::BPS, j1 - jj);
-                const uint32_t slot = it % NSTAGES;
-                if (it >= NSTAGES) {
-                    ok = mbar_wait_bounded(bar_empty + 8 * slot, ((it / NSTAGES) - 1) & 1);
-                    if (!ok) { raise_flag(p.flags, kFlagTimeout); break; }
-                }
-                const uint32_t full = bar_full + 8 * slot;
-                mbar_arrive_expect_tx(full, (uint32_t)(nb * 2 * C::TILE));
-                const uint32_t dK = sbase + slot * C::STAGE, dV = dK + C::STAGE_KV;
-                for (int b = 0; b < nb; ++b) {
-                    int pb = __ldg(bt + jj + b);
-                    if (pb < 0 || pb >= p.num_blocks) {
-                        raise_flag(p.flags, kFlagBlockId);
-                        pb = 0;
+            int jc = cur.j;
+            int pb_next = jc + lane < j1 ? __ldg(bt + jc + lane) : 0;
+            while (jc < j1 && ok) {
+                const int pb_cur = pb_next;
+                const int jn = jc + 32;
+                pb_next = jn + lane < j1 ? __ldg(bt + jn + lane) : 0;
+                const int chunk_end = min(j1, jn);
+                for (int jj = jc; jj < chunk_end; jj += C::BPS) {
+                    const int nb = min(C::BPS, j1 - jj);
+                    const uint32_t slot = it % NSTAGES;
+                    if (lane == 0 && it >= (uint32_t)NSTAGES)
+                        ok = mbar_wait_bounded(bar_empty + 8 * slot, ((it / NSTAGES) - 1) & 1);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    const uint32_t full = bar_full + 8 * slot;
+                    if (lane == 0) mbar_arrive_expect_tx(full, (uint32_t)(nb * 2 * C::TILE));
+                    const uint32_t dK = sbase + slot * C::STAGE, dV = dK + C::STAGE_KV;
+#pragma unroll
+                    for (int b = 0; b < C::BPS; ++b) {
+                        int pb = __shfl_sync(0xffffffffu, pb_cur, (jj - jc + b) & 31);
+                        if (b < nb && lane == 0) {
+                            if (pb < 0 || pb >= p.num_blocks) {
+                                raise_flag(p.flags, kFlagBlockId);
+                                pb = 0;
+                            }
+                            const int32_t row = pb * Hkv + cur.h;
+                            tma_load_4d(dK + b * C::TILE, &tmK, full, 0, 0, 0, row);
+                            tma_load_4d(dV + b * C::TILE, &tmV, full, 0, 0, 0, row);
+                        }
                     }
-                    const int32_t row = pb * Hkv + cur.h;
-                    tma_load_4d(dK + b * C::TILE, &tmK, full, 0, 0, 0, row);
-                    tma_load_4d(dV + b * C::TILE, &tmV, full, 0, 0, 0, row);
+                    ++it;
                 }
-                ++it;
+                jc = jn;
             }
             cur.u += j1 - cur.j;
             next_unit<BS>(cur, p);
         }
-        // drain: every issued stage must land before the CTA may exit
-        const uint32_t first = it > NSTAGES ? it - NSTAGES : 0;
-        for (uint32_t k = first; k < it; ++k)
-            if (!mbar_wait_bounded(bar_full + 8 * (k % NSTAGES), (k / NSTAGES) & 1, 200000000ull))
-                raise_flag(p.flags, kFlagTimeout);
+        if (!ok && lane == 0) raise_flag(p.flags, kFlagTimeout);
+        if (lane == 0) {
+            // the terminal descriptor needs the slot of segment sit - NSEG back
+            const uint32_t slot = sit % C::NSEG;
+            bool free_slot = true;
+            if (sit >= (uint32_t)C::NSEG)
+                free_slot = mbar_wait_bounded(seg_empty + 8 * slot, ((sit / C::NSEG) - 1) & 1);
+            // drain: every issued copy must land before the CTA may exit.  Each
+            // slot waited on here has no later arrival, so its parity is exact;
+            // segment sit - NSEG is skipped once the consumers released its
+            // slot (they had read its query rows, so that copy had landed).
+            const uint32_t first = it > NSTAGES ? it - NSTAGES : 0;
+            for (uint32_t k = first; k < it; ++k)
+                if (!mbar_wait_bounded(bar_full + 8 * (k % NSTAGES), (k / NSTAGES) & 1,
+                                       200000000ull))
+                    raise_flag(p.flags, kFlagTimeout);
+            uint32_t qfirst = sit > C::NSEG ? sit - C::NSEG : 0;
+            if (free_slot && sit >= (uint32_t)C::NSEG) qfirst = sit - C::NSEG + 1;
+            for (uint32_t k = qfirst; k < sit; ++k)
+                if (!mbar_wait_bounded(seg_full + 8 * (k % C::NSEG), (k / C::NSEG) & 1,
+                                       200000000ull))
+                    raise_flag(p.flags, kFlagTimeout);
+            // terminal descriptor (also after a timeout, so that the consumers stop)
+            if (free_slot) {
+                segs[slot].terminal = 1;
+                mbar_arrive(seg_full + 8 * slot);
+            }
+        }
         return;
     }
 
     // ==================== consumers (warps 0..3) ===========================
     const int gid = lane >> 2, t4 = lane & 3;
-    uint32_t it = 0;
+    uint32_t it = 0, sit = 0;
 
-    while (cur.u < u1) {
-        const int j0 = cur.j;
-        const int j1 = (int)min((long long)cur.n, cur.j + (u1 - cur.u));
-        const int s = cur.s, h = cur.h, ctx = cur.ctx;
-        const bool whole = (j0 == 0 && j1 == cur.n);
+    for (;;) {
+        // ---- next segment: descriptor + query fragments from shared memory
+        const uint32_t qs = sit % C::NSEG;
+        const bool seg_ok = mbar_wait_bounded(seg_full + 8 * qs, (sit / C::NSEG) & 1);
+        if (!seg_ok) raise_flag(p.flags, kFlagTimeout);
+        const uint32_t da = sSeg + qs * (uint32_t)sizeof(SegDesc);
+        const long long useg = lds64(da + offsetof(SegDesc, u));
+        const int s = (int)lds32(da + offsetof(SegDesc, s));
+        const int h = (int)lds32(da + offsetof(SegDesc, h));
+        const int j0 = (int)lds32(da + offsetof(SegDesc, j0));
+        const int j1 = (int)lds32(da + offsetof(SegDesc, j1));
+        const int nunit = (int)lds32(da + offsetof(SegDesc, n));
+        const int ctx = (int)lds32(da + offsetof(SegDesc, ctx));
+        const int terminal = (int)lds32(da + offsetof(SegDesc, terminal));
+        const float ksc = __uint_as_float(lds32(da + offsetof(SegDesc, ksc)));
+        const float vsc = __uint_as_float(lds32(da + offsetof(SegDesc, vsc)));
+        if (named_bar_sync_or(kBarConsumers, kConsumers, !seg_ok || terminal)) return;
+        const bool whole = (j0 == 0 && j1 == nunit);
 
-        // ---- query fragments (B operand, Q^T[d][head]) for this unit ----
+        // query fragments (B operand, Q^T[d][head]) from the slot
         uint32_t qf[C::KSTEPS][NT][2];
         {
-            const uint16_t *qb = p.q + ((long long)s * p.num_q_heads + (long long)h * g) * D;
+            const uint32_t qb = sQ + qs * C::QSLOT;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const int head = nt * 8 + gid;
                 const bool live = head < g;
-                const uint32_t *qr = reinterpret_cast<const uint32_t *>(qb + (live ? head : 0) * D);
+                const uint32_t qr = qb + (live ? head : 0) * D * 2;
 #pragma unroll
                 for (int k = 0; k < C::KSTEPS; ++k) {
                     uint32_t b0, b1;
                     if (!FP8) {   // k index 2t, 2t+1 | 2t+8, 2t+9  <->  same d
-                        b0 = __ldg(qr + (16 * k + 2 * t4) / 2);
-                        b1 = __ldg(qr + (16 * k + 8 + 2 * t4) / 2);
+                        b0 = lds32(qr + (16 * k + 2 * t4) * 2);
+                        b1 = lds32(qr + (16 * k + 8 + 2 * t4) * 2);
                     } else {      // k index permuted to d = 16k + 4t + {0,1 | 2,3}
-                        b0 = bf16x2_to_f16x2(__ldg(qr + (16 * k + 4 * t4) / 2));
-                        b1 = bf16x2_to_f16x2(__ldg(qr + (16 * k + 4 * t4 + 2) / 2));
+                        b0 = bf16x2_to_f16x2(lds32(qr + (16 * k + 4 * t4) * 2));
+                        b1 = bf16x2_to_f16x2(lds32(qr + (16 * k + 4 * t4 + 2) * 2));
                     }
                     qf[k][nt][0] = live ? b0 : 0u;
                     qf[k][nt][1] = live ? b1 : 0u;
                 }
             }
         }
-        float sl2 = p.scale_log2, vsc = 1.f;
-        if (FP8) {
-            sl2 *= __ldg(p.k_scale + h);
-            vsc = __ldg(p.v_scale + h);
-        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(seg_empty + 8 * qs);   // the slot may be refilled
+        ++sit;
+
+        const float sl2 = p.scale_log2 * ksc;
 
         float m_run[NT][2], l_run[NT][2];
-        float o_acc[C::MT][NT][4];
+        float o_hi[C::MT][NT][4], o_lo[C::MT][NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             m_run[nt][0] = m_run[nt][1] = -INFINITY;
             l_run[nt][0] = l_run[nt][1] = 0.f;
 #pragma unroll
             for (int mt = 0; mt < C::MT; ++mt)
-                o_acc[mt][nt][0] = o_acc[mt][nt][1] = o_acc[mt][nt][2] = o_acc[mt][nt][3] = 0.f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) o_hi[mt][nt][e] = o_lo[mt][nt][e] = 0.f;
         }
 
+        bool abort = false;
         for (int jj = j0; jj < j1; jj += C::BPS) {
             const int nb = min(C::BPS, j1 - jj);
             const int n_valid = min(ctx - jj * BS, nb * BS);
@@ -360,10 +557,12 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             if (!ok) raise_flag(p.flags, kFlagTimeout);
             const uint32_t sK = sbase + slot * C::STAGE, sV = sK + C::STAGE_KV;
 
-            // ---- S^T = K . Q^T for this warp's 16 tokens ----------------
-            float sacc[NT][4];
+            // ---- S^T = K . Q^T for this warp's 16 tokens (two MMA chains) --
+            float sacc[NT][4], sac2[NT][4];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sacc[nt][e] = sac2[nt][e] = 0.f;
             if (16 * warp < n_valid) {
                 if (!FP8) {
                     const int mi = lane >> 3;
@@ -378,8 +577,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                         uint32_t a0, a1, a2, a3;
                         ldsm_x4(addr, a0, a1, a2, a3);
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
-                            mma_bf16(sacc[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
+                        for (int nt = 0; nt < NT; ++nt) {
+                            if (k & 1) mma_bf16(sac2[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
+                            else       mma_bf16(sacc[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
+                        }
                     }
                 } else {
                     const int tok0 = 16 * warp + gid, tok1 = tok0 + 8;
@@ -388,16 +589,17 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     const uint32_t base1 = sK + (tok1 / BS) * C::TILE + r1 * 128 + 4 * t4;
 #pragma unroll
                     for (int k = 0; k < C::KSTEPS; ++k) {
-                        uint32_t w0, w1;
-                        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w0) : "r"(base0 + ((k ^ (r0 & 7)) << 4)));
-                        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w1) : "r"(base1 + ((k ^ (r1 & 7)) << 4)));
+                        const uint32_t w0 = lds32(base0 + ((k ^ (r0 & 7)) << 4));
+                        const uint32_t w1 = lds32(base1 + ((k ^ (r1 & 7)) << 4));
                         const uint32_t a0 = e4m3x2_to_f16x2(w0 & 0xffffu);
                         const uint32_t a2 = e4m3x2_to_f16x2(w0 >> 16);
                         const uint32_t a1 = e4m3x2_to_f16x2(w1 & 0xffffu);
                         const uint32_t a3 = e4m3x2_to_f16x2(w1 >> 16);
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
-                            mma_f16(sacc[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
+                        for (int nt = 0; nt < NT; ++nt) {
+                            if (k & 1) mma_f16(sac2[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
+                            else       mma_f16(sacc[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
+                        }
                     }
                 }
             }
@@ -410,7 +612,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 for (int e = 0; e < 4; ++e) {
                     const int tok = 16 * warp + gid + (e >> 1) * 8;
                     const int head = nt * 8 + 2 * t4 + (e & 1);
-                    sacc[nt][e] = (tok < n_valid && head < g) ? sacc[nt][e] * sl2 : -INFINITY;
+                    const float v = sacc[nt][e] + sac2[nt][e];
+                    sacc[nt][e] = (tok < n_valid && head < g) ? v * sl2 : -INFINITY;
                 }
                 mx[nt][0] = fmaxf(sacc[nt][0], sacc[nt][2]);
                 mx[nt][1] = fmaxf(sacc[nt][1], sacc[nt][3]);
@@ -487,18 +690,18 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             }
             // all consumers agree on whether any of them timed out
-            const bool abort = named_bar_sync_or(kBarConsumers, kConsumers, !ok);
+            abort = named_bar_sync_or(kBarConsumers, kConsumers, !ok);
 
             // ---- O^T += V^T . P^T for this warp's D/4 dims ------------------
 #pragma unroll
             for (int mt = 0; mt < C::MT; ++mt)
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    o_acc[mt][nt][0] *= alpha[nt][0];
-                    o_acc[mt][nt][1] *= alpha[nt][1];
-                    o_acc[mt][nt][2] *= alpha[nt][0];
-                    o_acc[mt][nt][3] *= alpha[nt][1];
-                }
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        o_hi[mt][nt][e] *= alpha[nt][e & 1];
+                        o_lo[mt][nt][e] *= alpha[nt][e & 1];
+                    }
 #pragma unroll
             for (int kk = 0; kk < kStageTokens / 16; ++kk) {
                 if (16 * kk >= n_valid) break;
@@ -532,8 +735,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                         ldsm_x4_t(addr, a0, a1, a2, a3);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
-                            mma_bf16(o_acc[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
-                            mma_bf16(o_acc[mt][nt], a0, a1, a2, a3, pl[nt][0], pl[nt][1]);
+                            mma_bf16(o_hi[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+                            mma_bf16(o_lo[mt][nt], a0, a1, a2, a3, pl[nt][0], pl[nt][1]);
                         }
                     }
                 } else {
@@ -545,9 +748,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     for (int q = 0; q < 4; ++q) {
                         const int tok = 16 * kk + 2 * t4 + (q & 1) + (q >> 1) * 8;
                         const int row = tok % BS;
-                        const uint32_t a = sV + (tok / BS) * C::TILE + row * 128 +
-                                           ((chunk ^ (row & 7)) << 4) + 4 * (gid & 3);
-                        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(wv[q]) : "r"(a));
+                        wv[q] = lds32(sV + (tok / BS) * C::TILE + row * 128 +
+                                      ((chunk ^ (row & 7)) << 4) + 4 * (gid & 3));
                     }
 #pragma unroll
                     for (int mt = 0; mt < C::MT; ++mt) {
@@ -560,15 +762,16 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                         const uint32_t a3 = e4m3x2_to_f16x2(y >> 16);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt)
-                            mma_f16(o_acc[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+                            mma_f16(o_hi[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
                     }
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_empty + 8 * slot);
             ++it;
-            if (abort) return;   // uniform over the consumers; the producer drains
+            if (abort) break;
         }
+        if (abort) return;   // uniform over the consumers; the producer drains
 
         // ---- finish the segment ---------------------------------------------
 #pragma unroll
@@ -607,7 +810,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     for (int e = 0; e < 4; ++e) {
                         const int head = nt * 8 + 2 * t4 + (e & 1);
                         if (head < g) {
-                            const float v = o_acc[mt][nt][e] * inv_l[nt][e & 1];
+                            const float v = (o_hi[mt][nt][e] + o_lo[mt][nt][e]) * inv_l[nt][e & 1];
                             p.out[(row0 + head) * D + dim_of(mt, e)] =
                                 __bfloat16_as_ushort(__float2bfloat16_rn(v));
                         }
@@ -623,7 +826,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             }
         } else {
             // partial: slot 2c for the CTA's first segment, 2c+1 for its last
-            const bool first_seg = (cur.u == u0);
+            const bool first_seg = (useg == u0);
             const long long slot = 2 * cta + (first_seg ? 0 : 1);
             float *op = p.o_part + slot * g * D;
 #pragma unroll
@@ -633,7 +836,9 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int head = nt * 8 + 2 * t4 + (e & 1);
-                        if (head < g) op[head * D + dim_of(mt, e)] = o_acc[mt][nt][e] * inv_l[nt][e & 1];
+                        if (head < g)
+                            op[head * D + dim_of(mt, e)] =
+                                (o_hi[mt][nt][e] + o_lo[mt][nt][e]) * inv_l[nt][e & 1];
                     }
             if (warp == 0 && gid == 0) {
 #pragma unroll
@@ -647,8 +852,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             __threadfence();
             named_bar_sync(kBarConsumers, kConsumers);
             // unit tile range [ua, ub) and the CTAs that share it
-            const long long ua = cur.u - j0;   // flattened index of tile (s, h, 0)
-            const long long ub = ua + cur.n;
+            const long long ua = useg - j0;   // flattened index of tile (s, h, 0)
+            const long long ub = ua + nunit;
             const long long c_first = cta_of(ua, U, G), c_last = cta_of(ub - 1, U, G);
             if (tid == 0) {
                 const int prev = atomicAdd(p.counters + (long long)s * Hkv + h, 1);
@@ -657,32 +862,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             named_bar_sync(kBarConsumers, kConsumers);
             if (misc->is_last) {
                 __threadfence();
-                for (int e = tid; e < g * D; e += kConsumers) {
-                    const int head = e / D, d = e % D;
-                    float M = -INFINITY;
-                    for (long long c = c_first; c <= c_last; ++c) {
-                        const long long sl = 2 * c + ((ua <= c * U / G) ? 0 : 1);
-                        M = fmaxf(M, __ldcg(p.lse_part + sl * g + head));
-                    }
-                    const float Mu = M == -INFINITY ? 0.f : M;
-                    float W = 0.f, acc = 0.f;
-                    for (long long c = c_first; c <= c_last; ++c) {
-                        const long long sl = 2 * c + ((ua <= c * U / G) ? 0 : 1);
-                        const float w = ex2(__ldcg(p.lse_part + sl * g + head) - Mu);
-                        W += w;
-                        acc += w * __ldcg(p.o_part + (sl * g + head) * D + d);
-                    }
-                    p.out[(row0 + head) * D + d] =
-                        __bfloat16_as_ushort(__float2bfloat16_rn(W > 0.f ? acc / W : 0.f));
-                    if (p.lse_out && d == 0)
-                        p.lse_out[row0 + head] = W > 0.f ? (M + log2f(W)) * kLn2 : -INFINITY;
-                }
+                merge_unit<D>(p, ua, U, G, c_first, c_last, row0, g);
                 if (tid == 0) p.counters[(long long)s * Hkv + h] = 0;
             }
         }
-
-        cur.u += j1 - j0;
-        next_unit<BS>(cur, p);
     }
 }
 

@@ -17,11 +17,11 @@ struct DecodeLaunchArgs {
     cudaStream_t stream;
 };
 
-// Shared-memory pipeline depth per family: about 96-192 KB of K/V in flight
-// per CTA.
+// Shared-memory pipeline depth per family: 96 KB of K/V stages per CTA for
+// head_dim 128 (two CTAs per SM), 192 KB for head_dim 256 (one per SM).
 template <int D, bool FP8>
 struct Stages {
-    static constexpr int value = FP8 ? 6 : (D == 128 ? 4 : 3);
+    static constexpr int value = FP8 ? 6 : 3;
 };
 
 template <int D, int BS, int NT, bool FP8>
