@@ -1,5 +1,6 @@
-"""Benchmark: one paged GQA decode step (kv_append + paged_decode_attention)
-on the Llama-3-8B-shaped workload (64 sequences, context U[512, 4096], 32 q /
+"""Benchmark: one paged GQA decode step (kv_append + paged_decode_attention,
+fused into one launch by pgd_decode_step; --unfused times the two calls) on
+the Llama-3-8B-shaped workload (64 sequences, context U[512, 4096], 32 q /
 8 KV heads, head_dim 128, block_size 16, bf16 KV, 64 new tokens appended).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -183,8 +184,16 @@ def run_ours(args, rank, world, local_rank):
     out = torch.empty_like(q)
     mcl = w.max_context_len
     stream = torch.cuda.current_stream()
+    # a decode step whose appended tokens are each sequence's newest token runs
+    # as one fused launch (pgd_decode_step); --unfused times append + decode
+    fused = has_app and not args.unfused and len(w.slot_mapping) == w.num_seqs
 
     def step(q_, kn_, vn_, sl_, bt_, cl_, out_):
+        if fused:
+            pgd.decode_step(q_, kn_, vn_, k, v, bt_, cl_, w.num_q_heads, w.num_kv_heads,
+                            w.head_dim, w.block_size, w.scale, out_, max_context_len=mcl,
+                            k_scale=ks, v_scale=vs, stream=stream)
+            return
         if has_app:
             pgd.kv_append(kn_, vn_, sl_, k, v, stream=stream)
         pgd.paged_decode_attention(q_, k, v, bt_, cl_, w.num_q_heads, w.num_kv_heads,
@@ -202,10 +211,26 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     assert pgd.get_device_error() == 0
 
-    # ---- timed region: K steps, device time, decode launches timed too -------
+    def decode_only():
+        if fused:
+            pgd.decode_step(q, kn, vn, k, v, bt, cl, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                            w.block_size, w.scale, out, max_context_len=mcl, k_scale=ks,
+                            v_scale=vs, stream=stream)
+        else:
+            pgd.paged_decode_attention(q, k, v, bt, cl, w.num_q_heads, w.num_kv_heads,
+                                       w.head_dim, w.block_size, w.scale, out,
+                                       max_context_len=mcl, k_scale=ks, v_scale=vs,
+                                       stream=stream)
+
+    # ---- timed region: K back-to-back steps, device time ---------------------
+    # No event sits between launches (an event between two launches stops the
+    # next launch from overlapping its set-up with the previous one's tail).
+    # With one launch per step the decode kernel's average launch duration is
+    # this region's time / K; the unfused mode brackets each decode launch.
     K = args.steps
-    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(K)]
+    single = fused or not has_app          # one launch per step
+    ev_dec = [] if single else [(torch.cuda.Event(enable_timing=True),
+                                 torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     clocks = ClockSampler(local_rank) if not args.no_clocks else None
     if clocks:
         clocks.start()
@@ -216,12 +241,12 @@ def run_ours(args, rank, world, local_rank):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(K):
-        if has_app:
-            pgd.kv_append(kn, vn, sl, k, v, stream=stream)
+        if single:
+            decode_only()
+            continue
+        pgd.kv_append(kn, vn, sl, k, v, stream=stream)
         ev_dec[i][0].record(stream)
-        pgd.paged_decode_attention(q, k, v, bt, cl, w.num_q_heads, w.num_kv_heads, w.head_dim,
-                                   w.block_size, w.scale, out, max_context_len=mcl,
-                                   k_scale=ks, v_scale=vs, stream=stream)
+        decode_only()
         ev_dec[i][1].record(stream)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -229,9 +254,20 @@ def run_ours(args, rank, world, local_rank):
     t_end = time.time()
     clk = clocks.stop(t_begin, t_end) if clocks else None
     ms_total = e0.elapsed_time(e1)
-    dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
-    dec_avg_ms = sum(dec_ms) / len(dec_ms)
+    if single:
+        dec_avg_ms = ms_total / K
+    else:
+        dec_avg_ms = sum(a.elapsed_time(b) for a, b in ev_dec) / K
     flags = pgd.get_device_error()
+    # for reference: the same launch bracketed by its own events, one at a time
+    iso = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(min(K, 50))]
+    for a_, b_ in iso:
+        a_.record(stream)
+        decode_only()
+        b_.record(stream)
+    torch.cuda.synchronize()
+    iso_ms = sum(a_.elapsed_time(b_) for a_, b_ in iso) / len(iso)
 
     # ---- end to end through the public API with host buffers ----------------
     hq = to_dev(w.q, pin=True)
@@ -280,7 +316,7 @@ def run_ours(args, rank, world, local_rank):
     value = world * step_bytes / (ms_step * 1e-3) / 1e9
     e2e_value = world * step_bytes / (e2e_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
-    dec_bytes = ab["decode_total"]
+    dec_bytes = ab["step_total"] if fused else ab["decode_total"]
     achieved = dec_bytes / (dec_avg_ms * 1e-3) / 1e9
 
     cpu = None
@@ -302,19 +338,25 @@ def run_ours(args, rank, world, local_rank):
             "config": cfg,
             "pct_of_measured_hbm": round(100 * value / world / peak, 1),
             "pct_of_nominal_8tbs": round(100 * value / world / 8000.0, 1),
-            "roofline": {"bound": "hbm", "kernel": "paged_decode_kernel",
+            "roofline": {"bound": "hbm",
+                         "kernel": "paged_decode_kernel" + (" (fused append)" if fused else ""),
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_kind == "measured" else "fallback 6.65 TB/s",
                          "algorithmic_bytes_per_launch": dec_bytes,
                          "avg_launch_us": round(dec_avg_ms * 1e3, 2),
+                         "launch_timing": "timed region / K (one launch per step, "
+                                          "back to back)" if single else
+                                          "events around each decode launch",
+                         "isolated_launch_us": round(iso_ms * 1e3, 2),
                          "traffic": recorded_traffic(args.workload)},
             "e2e": {"value": round(e2e_value, 1), "unit": "GB/s",
                     "us_per_step": round(e2e_ms * 1e3, 2),
                     "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
                     "steps": Ke},
-            "gpu_launches": K * (2 if has_app else 1),
+            "gpu_launches": K * (2 if has_app and not fused else 1),
+            "fused_step": fused,
             "clocks": clk,
             "device_flags": flags,
             "cpu_baseline": cpu,
@@ -430,6 +472,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--unfused", action="store_true",
+                    help="time kv_append and the decode as two launches")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

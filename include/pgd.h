@@ -180,6 +180,33 @@ pgd_status pgd_paged_decode_attention(
     void *workspace, size_t workspace_bytes, int32_t num_ctas, void *stream);
 
 /*
+ * pgd_decode_step -- one whole decode step in one launch: the KV append of
+ * each sequence's newest token ("batching and attention" 3.4: the new K/V
+ * row goes to its slot in the sequence's last block) fused with the decode
+ * attention of pgd_paged_decode_attention.  The result equals
+ * pgd_kv_append(k_new, v_new, slots) followed by pgd_paged_decode_attention,
+ * with slots[s] = block_table[s][(n-1)/block_size] * block_size +
+ * (n-1) % block_size, n = context_lens[s] (the count already includes the new
+ * token; sequences with n = 0 append nothing).
+ *
+ *   k_new, v_new  device [num_seqs][num_kv_heads][head_dim] in the cache type
+ *                 (bf16 or E4M3 bytes), 16-byte aligned
+ *   k_cache, v_cache  written at those slots, read everywhere else
+ *   all other arguments as pgd_paged_decode_attention.
+ * The CTA that reads a sequence's last tile for one KV head also writes that
+ * head's new row into it, before reading it, so no other launch is needed.
+ */
+pgd_status pgd_decode_step(
+    const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+    const int32_t *block_table, int32_t max_blocks_per_seq,
+    const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t num_blocks, float scale, pgd_kv_dtype kv_dtype,
+    const float *k_scale, const float *v_scale,
+    void *out, float *lse_out,
+    void *workspace, size_t workspace_bytes, int32_t num_ctas, void *stream);
+
+/*
  * pgd_paged_decode_attention_noalloc -- the same decode step as
  * pgd_paged_decode_attention, for callers that must not have the library
  * allocate device memory: a serving engine that has reserved nearly all HBM

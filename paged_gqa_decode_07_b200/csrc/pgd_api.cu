@@ -222,13 +222,21 @@ size_t pgd_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t
     return ws_layout(num_q_heads / num_kv_heads, head_dim, grid).total;
 }
 
-pgd_status pgd_paged_decode_attention(
-    const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
-    int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
-    int32_t max_context_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
-    int32_t block_size, int32_t num_blocks, float scale, pgd_kv_dtype kv_dtype,
-    const float *k_scale, const float *v_scale, void *out, float *lse_out, void *workspace,
-    size_t workspace_bytes, int32_t num_ctas, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared body of pgd_paged_decode_attention and pgd_decode_step (library
+// or caller workspace; k_new / v_new non-null selects the fused append).
+pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *block_table, int32_t max_blocks_per_seq,
+                       const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
+                       int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                       int32_t block_size, int32_t num_blocks, float scale,
+                       pgd_kv_dtype kv_dtype, const float *k_scale, const float *v_scale,
+                       const void *k_new, const void *v_new, void *out, float *lse_out,
+                       void *workspace, size_t workspace_bytes, int32_t num_ctas,
+                       void *stream) {
     // ---- host-side checks (nothing is enqueued on failure) ------------------
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
         max_blocks_per_seq <= 0 || max_context_len < 0 || num_ctas < 0)
@@ -253,6 +261,8 @@ pgd_status pgd_paged_decode_attention(
         (workspace && !aligned(workspace, 16)))
         return PGD_ERR_INVALID_ARG;
     if (!workspace && workspace_bytes) return PGD_ERR_INVALID_ARG;
+    if ((k_new == nullptr) != (v_new == nullptr)) return PGD_ERR_INVALID_ARG;
+    if (k_new && (!aligned(k_new, 16) || !aligned(v_new, 16))) return PGD_ERR_INVALID_ARG;
 
     DeviceState *d = nullptr;
     pgd_status st = device_state(&d);
@@ -319,6 +329,10 @@ pgd_status pgd_paged_decode_attention(
     p.context_lens = context_lens;
     p.k_scale = k_scale;
     p.v_scale = v_scale;
+    p.k_new = static_cast<const uint8_t *>(k_new);
+    p.v_new = static_cast<const uint8_t *>(v_new);
+    p.k_cache = static_cast<uint8_t *>(const_cast<void *>(k_cache));
+    p.v_cache = static_cast<uint8_t *>(const_cast<void *>(v_cache));
     p.counters = d->counters;
     p.lse_part = reinterpret_cast<float *>(ws + lay.lse);
     p.o_part = reinterpret_cast<float *>(ws + lay.opart);
@@ -334,6 +348,37 @@ pgd_status pgd_paged_decode_attention(
     a.stream = s;
     cudaError_t e = var.launch(a);
     return e == cudaSuccess ? PGD_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+pgd_status pgd_paged_decode_attention(
+    const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+    int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
+    int32_t max_context_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t num_blocks, float scale, pgd_kv_dtype kv_dtype,
+    const float *k_scale, const float *v_scale, void *out, float *lse_out, void *workspace,
+    size_t workspace_bytes, int32_t num_ctas, void *stream) {
+    return decode_impl(q, k_cache, v_cache, block_table, max_blocks_per_seq, context_lens,
+                       num_seqs, max_context_len, num_q_heads, num_kv_heads, head_dim,
+                       block_size, num_blocks, scale, kv_dtype, k_scale, v_scale, nullptr,
+                       nullptr, out, lse_out, workspace, workspace_bytes, num_ctas, stream);
+}
+
+pgd_status pgd_decode_step(
+    const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+    const int32_t *block_table, int32_t max_blocks_per_seq, const int32_t *context_lens,
+    int32_t num_seqs, int32_t max_context_len, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
+    pgd_kv_dtype kv_dtype, const float *k_scale, const float *v_scale, void *out,
+    float *lse_out, void *workspace, size_t workspace_bytes, int32_t num_ctas, void *stream) {
+    if (num_seqs > 0 && (!k_new || !v_new)) return PGD_ERR_INVALID_ARG;
+    return decode_impl(q, k_cache, v_cache, block_table, max_blocks_per_seq, context_lens,
+                       num_seqs, max_context_len, num_q_heads, num_kv_heads, head_dim,
+                       block_size, num_blocks, scale, kv_dtype, k_scale, v_scale, k_new, v_new,
+                       out, lse_out, workspace, workspace_bytes, num_ctas, stream);
 }
 
 pgd_status pgd_merge_partials(const float *o_part, const float *lse_part, int32_t num_parts,

@@ -18,14 +18,18 @@
 // otherwise it writes a partial (o, lse) and the CTA that completes the
 // unit's last share merges the partials by log-sum-exp.
 //
-// CTA = 4 consumer warps + 1 producer warp.  The producer is the only warp
-// that reads the inputs from global memory: it walks the segments, writes a
+// CTA = 4 consumer warps + 1 producer warp + 1 appender warp.  The producer
+// is the only warp that reads the inputs from global memory: it walks the
+// segments, writes a
 // descriptor for each into a small shared-memory ring together with the
 // unit's query rows (bulk copy), loads the block-table entries 32 at a time,
 // and issues one TMA tensor load per (block, KV head) tile of K and of V into
 // a ring of 64-token stages (128-byte swizzle, mbarrier completion).  Each
 // K/V tile is fetched once and used by all g query heads of the group
-// ("prefill and decode attention": GQA reuse).
+// ("prefill and decode attention": GQA reuse).  In a fused decode step the
+// appender warp writes each sequence's newest K/V row into the cache ahead of
+// the producer ("batching and attention" 3.4: the new token's slot), so the
+// append costs no extra launch.
 //
 // Per stage the consumers run a small tensor-core contraction per warp
 // (mma.sync m16n8k16, fp32 accumulate) with the roles transposed so that the
@@ -52,6 +56,13 @@ struct DecodeParams {
     const int32_t *context_lens;  // [B]
     const float *k_scale;         // [Hkv] (FP8 only)
     const float *v_scale;
+    // fused append (decode step): the K/V rows of each sequence's newest
+    // token, [B][Hkv][D] in the cache type, written to position ctx - 1
+    // before that tile is read; null when the caller appended already.
+    const uint8_t *k_new;
+    const uint8_t *v_new;
+    uint8_t *k_cache;             // raw cache pointers (fused append only)
+    uint8_t *v_cache;
     int32_t *counters;            // [B * Hkv], zero between calls
     float *o_part;                // [2 * grid][g][D]
     float *lse_part;              // [2 * grid][g], log2 domain
@@ -63,7 +74,8 @@ struct DecodeParams {
 
 constexpr int kConsumerWarps = 4;
 constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kThreads = kConsumers + 32;
+constexpr int kThreads = kConsumers + 64;   // + producer warp + appender warp
+constexpr int kAppSlots = 4;                // appender -> producer handoff ring
 constexpr int kStageTokens = 16 * kConsumerWarps;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kBarConsumers = 1;
@@ -100,7 +112,7 @@ struct DecodeCfg {
     static constexpr int OFF_RED = OFF_SEG + NSEG * (int)sizeof(SegDesc);
     static constexpr int OFF_LSUM = OFF_RED + kConsumerWarps * NP * 4;
     static constexpr int OFF_BAR = OFF_LSUM + kConsumerWarps * NP * 4;
-    static constexpr int NBARS = 2 * NSTAGES + 2 * NSEG;
+    static constexpr int NBARS = 2 * NSTAGES + 2 * NSEG + 2 * kAppSlots;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int MISC_BYTES = 256;
     static constexpr int SMEM = OFF_MISC + MISC_BYTES + 1024;   // + alignment slack
@@ -302,12 +314,20 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
     const uint32_t bar_empty = bar_full + NSTAGES * 8;
     const uint32_t seg_full = bar_empty + NSTAGES * 8;
     const uint32_t seg_empty = seg_full + C::NSEG * 8;
+    const uint32_t app_done = seg_empty + C::NSEG * 8;
+    const uint32_t app_free = app_done + kAppSlots * 8;
     const uint32_t sP = sbase + C::OFF_P;
     const uint32_t sQ = sbase + C::OFF_Q;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int B = p.num_seqs, Hkv = p.num_kv_heads, g = p.group;
     const long long cta = blockIdx.x;
+
+    // Programmatic dependent launch: let the next launch on the stream be
+    // scheduled now, and wait until the previous one has completed and its
+    // writes are visible before this grid reads anything from global memory.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (tid == 0) {
         for (int i = 0; i < NSTAGES; ++i) {
@@ -317,6 +337,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         for (int i = 0; i < C::NSEG; ++i) {
             mbar_init(seg_full + 8 * i, 1);
             mbar_init(seg_empty + 8 * i, kConsumerWarps);
+        }
+        for (int i = 0; i < kAppSlots; ++i) {
+            mbar_init(app_done + 8 * i, 1);
+            mbar_init(app_free + 8 * i, 1);
         }
         fence_mbar_init();
         misc->found = 0;
@@ -369,6 +393,65 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
     }
     __syncthreads();
 
+    if (warp == kConsumerWarps + 1) {
+        // ================= appender warp (fused append only) ===============
+        // Walks the same segments as the producer.  For each segment that
+        // holds its unit's last block it writes the newest token's K and V
+        // rows into the cache (position ctx - 1), orders those generic writes
+        // before async-proxy reads, and signals the producer, which waits for
+        // the signal before loading that block.  Only this CTA reads the
+        // unit's last tile, so no other CTA can see the row half-written.
+        if (p.k_new == nullptr) return;
+        Cursor cur;
+        cur.s = misc->s0;
+        cur.ctx = ctx_of<BS>(p, cur.s);
+        cur.n = nblk_of<BS>(cur.ctx);
+        {
+            const long long off = u0 - misc->pfx0;
+            cur.h = (int)(off / cur.n);
+            cur.j = (int)(off % cur.n);
+        }
+        cur.u = u0;
+        uint32_t ait = 0;
+        while (cur.u < u1) {
+            const int j1 = (int)min((long long)cur.n, cur.j + (u1 - cur.u));
+            if (j1 == cur.n) {
+                const uint32_t as = ait % kAppSlots;
+                bool ok = true;
+                if (lane == 0 && ait >= (uint32_t)kAppSlots)
+                    ok = mbar_wait_bounded(app_free + 8 * as, ((ait / kAppSlots) - 1) & 1);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) {
+                    if (lane == 0) raise_flag(p.flags, kFlagTimeout);
+                    return;
+                }
+                int pb = __ldg(p.block_table + (long long)cur.s * p.max_blocks_per_seq + cur.n - 1);
+                if (pb < 0 || pb >= p.num_blocks) {
+                    if (lane == 0) raise_flag(p.flags, kFlagBlockId);
+                    pb = 0;
+                }
+                const long long dst =
+                    (((long long)pb * Hkv + cur.h) * BS + (cur.ctx - 1) % BS) * C::ROW;
+                const long long src = ((long long)cur.s * Hkv + cur.h) * C::ROW;
+                constexpr int CH = C::ROW / 16;   // 16-byte chunks per row
+                for (int c = lane; c < 2 * CH; c += 32) {
+                    const bool isk = c < CH;
+                    const int off = 16 * (isk ? c : c - CH);
+                    const uint4 v =
+                        __ldg(reinterpret_cast<const uint4 *>((isk ? p.k_new : p.v_new) + src + off));
+                    *reinterpret_cast<uint4 *>((isk ? p.k_cache : p.v_cache) + dst + off) = v;
+                }
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(app_done + 8 * as);
+                ++ait;
+            }
+            cur.u += j1 - cur.j;
+            next_unit<BS>(cur, p);
+        }
+        return;
+    }
+
     if (warp == kConsumerWarps) {
         // ================= producer warp ====================================
         Cursor cur;
@@ -382,7 +465,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         }
         cur.u = u0;
         const uint32_t qbytes = (uint32_t)(g * D * 2);
-        uint32_t it = 0, sit = 0;
+        uint32_t it = 0, sit = 0, ait = 0;
         bool ok = true;
         while (cur.u < u1 && ok) {
             const int j1 = (int)min((long long)cur.n, cur.j + (u1 - cur.u));
@@ -413,6 +496,9 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 }
                 ++sit;
             }
+            // a segment that holds its unit's last block takes the appended
+            // row from the appender warp before that block is loaded
+            const bool app_seg = p.k_new != nullptr && j1 == cur.n;
             // -- K/V tiles, block ids fetched 32 at a time (one chunk ahead)
             const int32_t *bt = p.block_table + (long long)cur.s * p.max_blocks_per_seq;
             int jc = cur.j;
@@ -427,6 +513,13 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     const uint32_t slot = it % NSTAGES;
                     if (lane == 0 && it >= (uint32_t)NSTAGES)
                         ok = mbar_wait_bounded(bar_empty + 8 * slot, ((it / NSTAGES) - 1) & 1);
+                    if (app_seg && jj + nb == j1 && lane == 0 && ok) {
+                        // the appended row is in this stage: wait for its write
+                        const uint32_t as = ait % kAppSlots;
+                        ok = mbar_wait_bounded(app_done + 8 * as, (ait / kAppSlots) & 1);
+                        mbar_arrive(app_free + 8 * as);
+                        ++ait;
+                    }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     const uint32_t full = bar_full + 8 * slot;

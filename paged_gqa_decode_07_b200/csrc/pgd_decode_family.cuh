@@ -36,8 +36,19 @@ cudaError_t launch_decode(const DecodeLaunchArgs &a) {
     using C = DecodeCfg<D, BS, NT, FP8, NS>;
     cudaError_t e = ensure_smem_attr<D, BS, NT, FP8>();
     if (e != cudaSuccess) return e;
-    paged_decode_kernel<D, BS, NT, FP8, NS><<<a.grid, kThreads, C::SMEM, a.stream>>>(a.tmK, a.tmV, a.p);
-    return cudaGetLastError();
+    // programmatic dependent launch: the kernel waits (griddepcontrol.wait)
+    // for the previous work on the stream before its first global read
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(a.grid));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, paged_decode_kernel<D, BS, NT, FP8, NS>, a.tmK, a.tmV, a.p);
 }
 
 template <int D, int BS, int NT, bool FP8>

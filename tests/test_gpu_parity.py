@@ -215,3 +215,53 @@ def test_out_of_range_inputs_are_flagged_not_faulting():
     torch.cuda.synchronize()
     ref, _ = oracle_full(w)
     assert_close(to_f64(out), ref, "bf16", "after flags")
+
+
+# --------------------------------------------------------------------------- #
+# fused decode step: append of each sequence's newest token + decode, one launch
+# --------------------------------------------------------------------------- #
+def _step_payload(w):
+    """k_new / v_new [B][Hkv][D] for pgd_decode_step from the append payload
+    (one row per live sequence, zeros for empty ones)."""
+    live = [s for s in range(w.num_seqs) if w.context_lens[s] > 0]
+    kn = np.zeros((w.num_seqs,) + w.k_new.shape[1:], w.k_new.dtype)
+    vn = np.zeros_like(kn)
+    kn[live] = w.k_new
+    vn[live] = w.v_new
+    return kn, vn
+
+
+STEP_CASES = [  # (ctx, Hq, Hkv, D, bs, dtype, num_ctas)
+    ([1, 15, 16, 17, 200, 1000, 2049, 0, 333], 32, 8, 128, 16, "bf16", 0),
+    ([1, 15, 16, 17, 200, 1000, 2049, 0, 333], 32, 8, 128, 16, "bf16", 7),
+    ([700, 5, 3000, 64], 32, 2, 256, 32, "bf16", 0),
+    ([64, 900, 17, 4000, 1], 64, 8, 128, 16, "e4m3", 0),
+    ([65, 128, 129], 16, 2, 128, 64, "bf16", 3),
+]
+
+
+@pytest.mark.parametrize("ctx,Hq,Hkv,D,bs,dt,nctas", STEP_CASES,
+                         ids=[f"g{c[1] // c[2]}-D{c[3]}-bs{c[4]}-{c[5]}-n{c[6]}" for c in STEP_CASES])
+def test_fused_decode_step(ctx, Hq, Hkv, D, bs, dt, nctas):
+    from tests.gpu_helpers import dev_cache
+    w = make_case(ctx, Hq, Hkv, D, bs, dt, seed=200 + D + bs, append_last=True)
+    kn, vn = _step_payload(w)
+    # fused path
+    d1 = Dev(w)
+    lse1 = torch.empty((w.num_seqs, Hq), dtype=torch.float32, device="cuda")
+    out1 = pgd.decode_step(d1.q, dev_cache(kn), dev_cache(vn), d1.k, d1.v, d1.bt, d1.cl, Hq, Hkv,
+                           D, bs, w.scale, max_context_len=w.max_context_len, k_scale=d1.ks,
+                           v_scale=d1.vs, lse_out=lse1, num_ctas=nctas)
+    # two-launch path on a fresh copy
+    d2 = Dev(w)
+    d2.append()
+    out2, lse2 = d2.decode(num_ctas=nctas)
+    torch.cuda.synchronize()
+    ek, ev = oracle_caches(w)
+    assert np.array_equal(host_bits(d1.k), ek) and np.array_equal(host_bits(d1.v), ev)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    assert torch.equal(lse1, lse2)
+    ref, ref_lse = oracle_full(w)
+    got = to_f64(out1)
+    assert np.all(np.isfinite(got))
+    assert_close(got, ref, dt, "fused step")
