@@ -168,6 +168,17 @@ bool pick_variant(int D, int bs, int nt, bool fp8, Variant *v) {
 bool supported_block(int bs) { return bs == 16 || bs == 32 || bs == 64; }
 bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
 
+// Fixed cost of one (sequence, KV head) unit in a CTA (descriptor, query
+// rows, block-table fetch, first-tile latency, output) expressed as the K/V
+// bytes a CTA streams in the same time, about 2 us at 20 GB/s.  The batch is
+// cut by tiles + this many tile-equivalents per unit.
+constexpr long long kUnitOverheadBytes = 40 * 1024;
+
+int32_t unit_cost_tiles(int head_dim, int block_size, bool fp8) {
+    const long long tile_kv = 2LL * block_size * head_dim * (fp8 ? 1 : 2);
+    return static_cast<int32_t>((kUnitOverheadBytes + tile_kv - 1) / tile_kv);
+}
+
 }  // namespace
 
 extern "C" {
@@ -344,6 +355,7 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     p.group = g;
     p.num_blocks = num_blocks;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.unit_cost = unit_cost_tiles(head_dim, block_size, fp8);
     a.grid = static_cast<int>(grid);
     a.stream = s;
     cudaError_t e = var.launch(a);
@@ -601,6 +613,7 @@ extern "C" pgd_status pgd_paged_decode_attention_noalloc(
     p.group = g;
     p.num_blocks = num_blocks;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.unit_cost = unit_cost_tiles(head_dim, block_size, fp8);
     a.grid = static_cast<int>(grid);
     a.stream = s;
     e = var.launch(a);

@@ -70,6 +70,7 @@ struct DecodeParams {
     int32_t max_blocks_per_seq;
     int32_t num_seqs, num_q_heads, num_kv_heads, group, num_blocks;
     float scale_log2;             // softmax scale * log2(e)
+    int32_t unit_cost;            // work weight of a unit's fixed cost, in tiles
 };
 
 constexpr int kConsumerWarps = 4;
@@ -181,21 +182,29 @@ __device__ __forceinline__ long long block_scan(long long v, long long &total, M
     return v + before;
 }
 
-// The CTA that holds flattened tile x (ranges are [c*U/G, (c+1)*U/G), all
+// The CTA that holds work index x (ranges are [c*U/G, (c+1)*U/G), all
 // non-empty since G <= U).
 __device__ __forceinline__ long long cta_of(long long x, long long U, long long G) {
     return ((x + 1) * G - 1) / U;
 }
 
-// Walk state of the producer.
+// Work weight of one (sequence, KV head) unit of n tiles: its tiles plus a
+// fixed cost, so that a CTA given many short units gets fewer of them.
+__device__ __forceinline__ long long unit_weight(int n, int unit_cost) {
+    return n > 0 ? (long long)n + unit_cost : 0;
+}
+
+// Walk over the units of a CTA's work range (producer and appender).  Unit
+// (s, h) occupies work indices [a, a + w): its n tiles first, then the
+// fixed-cost slots, which hold no tiles.
 struct Cursor {
-    int s, h, j, n, ctx;
-    long long u;
+    int s, h, n, ctx;
+    long long a, w;
 };
 
 template <int BS>
 __device__ __forceinline__ void next_unit(Cursor &c, const DecodeParams &p) {
-    c.j = 0;
+    c.a += c.w;
     if (++c.h == p.num_kv_heads) {
         c.h = 0;
         for (++c.s; c.s < p.num_seqs; ++c.s) {
@@ -203,7 +212,21 @@ __device__ __forceinline__ void next_unit(Cursor &c, const DecodeParams &p) {
             c.n = nblk_of<BS>(c.ctx);
             if (c.n) break;
         }
+        c.w = unit_weight(c.n, p.unit_cost);
     }
+}
+
+template <int BS>
+__device__ __forceinline__ Cursor first_unit(const DecodeParams &p, int s0, long long pfx0,
+                                            long long u0) {
+    Cursor c;
+    c.s = s0;
+    c.ctx = ctx_of<BS>(p, s0);
+    c.n = nblk_of<BS>(c.ctx);
+    c.w = unit_weight(c.n, p.unit_cost);
+    c.h = (int)((u0 - pfx0) / c.w);
+    c.a = pfx0 + (long long)c.h * c.w;
+    return c;
 }
 
 __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uint32_t bytes,
@@ -352,7 +375,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
 
     // ---- prologue: total tiles and this CTA's range --------------------
     long long mine = 0;
-    for (int s = tid; s < B; s += kThreads) mine += nblk_of<BS>(ctx_of<BS>(p, s));
+    for (int s = tid; s < B; s += kThreads)
+        mine += unit_weight(nblk_of<BS>(ctx_of<BS>(p, s)), p.unit_cost);
     const long long U = block_sum(mine, misc) * Hkv;
     // CTAs beyond the tile count get no range, so every range is non-empty
     const long long G = min((long long)gridDim.x, U);
@@ -377,7 +401,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         long long base = 0;
         for (int sb = 0; sb < B; sb += kThreads) {
             const int s = sb + tid;
-            const long long wgt = s < B ? (long long)nblk_of<BS>(ctx_of<BS>(p, s)) * Hkv : 0;
+            const long long wgt =
+                s < B ? unit_weight(nblk_of<BS>(ctx_of<BS>(p, s)), p.unit_cost) * Hkv : 0;
             long long tot;
             const long long incl = block_scan(wgt, tot, misc);
             const long long excl = base + incl - wgt;
@@ -402,20 +427,12 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         // the signal before loading that block.  Only this CTA reads the
         // unit's last tile, so no other CTA can see the row half-written.
         if (p.k_new == nullptr) return;
-        Cursor cur;
-        cur.s = misc->s0;
-        cur.ctx = ctx_of<BS>(p, cur.s);
-        cur.n = nblk_of<BS>(cur.ctx);
-        {
-            const long long off = u0 - misc->pfx0;
-            cur.h = (int)(off / cur.n);
-            cur.j = (int)(off % cur.n);
-        }
-        cur.u = u0;
+        Cursor cur = first_unit<BS>(p, misc->s0, misc->pfx0, u0);
         uint32_t ait = 0;
-        while (cur.u < u1) {
-            const int j1 = (int)min((long long)cur.n, cur.j + (u1 - cur.u));
-            if (j1 == cur.n) {
+        for (; cur.a < u1; next_unit<BS>(cur, p)) {
+            const long long j0 = max(0LL, u0 - cur.a);
+            const int j1 = (int)min((long long)cur.n, u1 - cur.a);
+            if (j0 < j1 && j1 == cur.n) {
                 const uint32_t as = ait % kAppSlots;
                 bool ok = true;
                 if (lane == 0 && ait >= (uint32_t)kAppSlots)
@@ -446,29 +463,20 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 if (lane == 0) mbar_arrive(app_done + 8 * as);
                 ++ait;
             }
-            cur.u += j1 - cur.j;
-            next_unit<BS>(cur, p);
         }
         return;
     }
 
     if (warp == kConsumerWarps) {
         // ================= producer warp ====================================
-        Cursor cur;
-        cur.s = misc->s0;
-        cur.ctx = ctx_of<BS>(p, cur.s);
-        cur.n = nblk_of<BS>(cur.ctx);
-        {
-            const long long off = u0 - misc->pfx0;
-            cur.h = (int)(off / cur.n);
-            cur.j = (int)(off % cur.n);
-        }
-        cur.u = u0;
+        Cursor cur = first_unit<BS>(p, misc->s0, misc->pfx0, u0);
         const uint32_t qbytes = (uint32_t)(g * D * 2);
         uint32_t it = 0, sit = 0, ait = 0;
         bool ok = true;
-        while (cur.u < u1 && ok) {
-            const int j1 = (int)min((long long)cur.n, cur.j + (u1 - cur.u));
+        for (; cur.a < u1 && ok; next_unit<BS>(cur, p)) {
+            const int j0 = (int)max(0LL, u0 - cur.a);
+            const int j1 = (int)min((long long)cur.n, u1 - cur.a);
+            if (j0 >= j1) continue;   // the range holds only this unit's fixed-cost slots
             // -- descriptor and query rows of the segment
             {
                 const uint32_t slot = sit % C::NSEG;
@@ -478,10 +486,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 if (!ok) break;
                 if (lane == 0) {
                     SegDesc &d = segs[slot];
-                    d.u = cur.u;
+                    d.u = cur.a + j0;
                     d.s = cur.s;
                     d.h = cur.h;
-                    d.j0 = cur.j;
+                    d.j0 = j0;
                     d.j1 = j1;
                     d.n = cur.n;
                     d.ctx = cur.ctx;
@@ -501,7 +509,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             const bool app_seg = p.k_new != nullptr && j1 == cur.n;
             // -- K/V tiles, block ids fetched 32 at a time (one chunk ahead)
             const int32_t *bt = p.block_table + (long long)cur.s * p.max_blocks_per_seq;
-            int jc = cur.j;
+            int jc = j0;
             int pb_next = jc + lane < j1 ? __ldg(bt + jc + lane) : 0;
             while (jc < j1 && ok) {
                 const int pb_cur = pb_next;
@@ -542,8 +550,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 }
                 jc = jn;
             }
-            cur.u += j1 - cur.j;
-            next_unit<BS>(cur, p);
         }
         if (!ok && lane == 0) raise_flag(p.flags, kFlagTimeout);
         if (lane == 0) {
