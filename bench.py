@@ -152,6 +152,31 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- #
+# rank aggregation                                                            #
+# --------------------------------------------------------------------------- #
+def reduce_over_ranks(step_bytes: int, ms_step: float, e2e_ms: float, dec_ms: float,
+                      world: int, device=None) -> dict:
+    """Whole-job figures over all ranks: the bytes every rank moved in one step
+    are summed, each time is the maximum over ranks, and value = summed bytes
+    / max step time.  Works on any initialised process group (nccl with CUDA
+    tensors, gloo with CPU ones); with world == 1 it only divides."""
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        t = torch.tensor([ms_step, e2e_ms, dec_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, e2e_ms, dec_ms = t.tolist()
+        b = torch.tensor([float(step_bytes)], dtype=torch.float64, device=device)
+        dist.all_reduce(b, op=dist.ReduceOp.SUM)
+        total_bytes = b.item()
+    else:
+        total_bytes = float(step_bytes)
+    return {"ms_step": ms_step, "e2e_ms": e2e_ms, "dec_ms": dec_ms, "total_bytes": total_bytes,
+            "value": total_bytes / (ms_step * 1e-3) / 1e9,
+            "e2e_value": total_bytes / (e2e_ms * 1e-3) / 1e9}
+
+
+# --------------------------------------------------------------------------- #
 # our arm                                                                     #
 # --------------------------------------------------------------------------- #
 def run_ours(args, rank, world, local_rank):
@@ -163,7 +188,9 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = make_workload(args.workload, seed=rank)   # an independent batch per rank
+    # every rank runs its own batch: same shape (context lengths of seed 0),
+    # its own block permutation and values
+    w = make_workload(args.workload, seed=rank, shape_seed=0)
     ab = w.algorithmic_bytes()
 
     def to_dev(a, pin=False):
@@ -306,15 +333,11 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     e2e_ms = f0.elapsed_time(f1) / Ke
 
-    # ---- aggregate over ranks (max time) -------------------------------------
+    # ---- aggregate over ranks ----------------------------------------------------
     ms_step = ms_total / K
-    if world > 1:
-        t = torch.tensor([ms_step, e2e_ms, dec_avg_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, e2e_ms, dec_avg_ms = t.tolist()
-    step_bytes = ab["step_total"]
-    value = world * step_bytes / (ms_step * 1e-3) / 1e9
-    e2e_value = world * step_bytes / (e2e_ms * 1e-3) / 1e9
+    agg = reduce_over_ranks(ab["step_total"], ms_step, e2e_ms, dec_avg_ms, world, dev)
+    ms_step, e2e_ms, dec_avg_ms = agg["ms_step"], agg["e2e_ms"], agg["dec_ms"]
+    value, e2e_value = agg["value"], agg["e2e_value"]
     peak, peak_kind = measured_peak()
     dec_bytes = ab["step_total"] if fused else ab["decode_total"]
     achieved = dec_bytes / (dec_avg_ms * 1e-3) / 1e9

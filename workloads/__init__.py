@@ -258,8 +258,11 @@ def context_lens_for(name: str, seed: int = 0) -> np.ndarray:
     raise KeyError(name)
 
 
-def make_workload(name: str, seed: int = 0) -> Workload:
-    ctx = context_lens_for(name, seed)
+def make_workload(name: str, seed: int = 0, shape_seed: Optional[int] = None) -> Workload:
+    """The named workload.  `shape_seed` (default `seed`) draws the context
+    lengths; `seed` draws the block permutation and the values, so replicas
+    that share a shape_seed have the same shape and their own data."""
+    ctx = context_lens_for(name, seed if shape_seed is None else shape_seed)
     if name == "tiny":
         return make_case(ctx, 8, 2, 128, 16, "bf16", seed, pool=64, name=name)
     if name == "llama3_8b_decode":
