@@ -64,6 +64,11 @@ def configure(lib):
     lib.pgdo_paged_decode_tiled.argtypes = args + [i32, i32, P, P]
     lib.pgdo_merge_partials.restype = ctypes.c_int
     lib.pgdo_merge_partials.argtypes = [P, P, i32, i32, i32, P, P]
+    lib.pgdo_e4m3_from_double.restype = ctypes.c_uint8
+    lib.pgdo_e4m3_from_double.argtypes = [dbl]
+    lib.pgdo_encode_e4m3_array.argtypes = [P, P, i64]
+    lib.pgdo_kv_append_quant.restype = ctypes.c_int
+    lib.pgdo_kv_append_quant.argtypes = [P, P, P, i32, P, P, P, P, i32, i32, i32, i32]
     return lib
 
 
@@ -201,3 +206,28 @@ def merge_partials(o_part, lse_part):
     if rc:
         raise OracleError(f"pgdo_merge_partials rc={rc}")
     return out, lse
+
+
+def e4m3_from_double(x: np.ndarray) -> np.ndarray:
+    """Nearest E4M3 bytes (ties to even, saturating at +-448)."""
+    x = _c(x, np.float64)
+    out = np.empty(x.shape, np.uint8)
+    _load().pgdo_encode_e4m3_array(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def kv_append_quant(k_new, v_new, slot_mapping, k_cache, v_cache, k_scale, v_scale, block_size):
+    """bf16 rows (uint16 bits) [N][Hkv][D] -> E4M3 cache bytes; returns new
+    (k_cache, v_cache); inputs are not modified."""
+    k_cache = np.array(k_cache, dtype=np.uint8, copy=True, order="C")
+    v_cache = np.array(v_cache, dtype=np.uint8, copy=True, order="C")
+    kn, vn = _c(k_new, np.uint16), _c(v_new, np.uint16)
+    ks, vs = _c(k_scale, np.float32), _c(v_scale, np.float32)
+    slots = _c(slot_mapping, np.int64)
+    nb, hkv, bs, d = k_cache.shape
+    assert bs == block_size
+    rc = _load().pgdo_kv_append_quant(_ptr(kn), _ptr(vn), _ptr(slots), len(slots), _ptr(k_cache),
+                                      _ptr(v_cache), _ptr(ks), _ptr(vs), hkv, d, bs, nb)
+    if rc:
+        raise OracleError(f"pgdo_kv_append_quant rc={rc}")
+    return k_cache, v_cache

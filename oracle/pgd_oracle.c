@@ -92,6 +92,35 @@ double pgdo_e4m3_to_double(uint8_t bits)
     return sign ? -mag : mag;
 }
 
+/* Nearest E4M3 value to y, ties to the even mantissa, magnitudes above the
+ * largest finite value (448) saturating to +-448 and NaN giving 0x7F.  Written
+ * from the format: normal values (1 + m/8) * 2^(e-7) for e = 1..15 (S.1111.111
+ * excluded), subnormals m * 2^-9.  The default floating-point rounding mode
+ * (to nearest, ties to even) makes nearbyint the tie-to-even step. */
+uint8_t pgdo_e4m3_from_double(double y)
+{
+    if (isnan(y)) return 0x7F;
+    const int sign = signbit(y) ? 0x80 : 0;
+    const double a = fabs(y);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    if (a < ldexp(1.0, -6)) {                      /* subnormal range */
+        const int k = (int)nearbyint(ldexp(a, 9));  /* a / 2^-9, 0..8 */
+        return (uint8_t)(sign | (k == 8 ? 0x08 : k)); /* 8 * 2^-9 is the smallest normal */
+    }
+    int e2;
+    frexp(a, &e2);                                 /* a = f * 2^e2, f in [0.5, 1) */
+    int E = e2 - 1;                                /* a in [2^E, 2^(E+1)) */
+    int m = (int)nearbyint((ldexp(a, -E) - 1.0) * 8.0);
+    if (m == 8) { m = 0; ++E; }
+    if (E > 8 || (E == 8 && m == 7)) return (uint8_t)(sign | 0x7E);
+    return (uint8_t)(sign | ((E + 7) << 3) | m);
+}
+
+void pgdo_encode_e4m3_array(const double *src, uint8_t *dst, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) dst[i] = pgdo_e4m3_from_double(src[i]);
+}
+
 void pgdo_decode_bf16_array(const uint16_t *src, double *dst, int64_t n)
 {
     for (int64_t i = 0; i < n; ++i) dst[i] = pgdo_bf16_to_double(src[i]);
@@ -126,6 +155,44 @@ int pgdo_kv_append(const void *k_new, const void *v_new,
             int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * row;
             memcpy((char *)k_cache + dst, (const char *)k_new + src, (size_t)row);
             memcpy((char *)v_cache + dst, (const char *)v_new + src, (size_t)row);
+        }
+    }
+    return PGDO_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Quantising KV append: bf16 K/V rows of new tokens go into an FP8 E4M3     */
+/* cache ("attention kernels", "what to check": FP8 KV cache).  Each element */
+/* is divided by its KV head's fp32 scale in fp32 (the precision the kernel  */
+/* decides the code in), then rounded to the nearest E4M3 value (ties to     */
+/* even, saturating at +-448) by pgdo_e4m3_from_double.                      */
+/* ------------------------------------------------------------------------- */
+int pgdo_kv_append_quant(const uint16_t *k_new, const uint16_t *v_new,
+                         const int64_t *slot_mapping, int32_t num_tokens,
+                         uint8_t *k_cache, uint8_t *v_cache,
+                         const float *k_scale, const float *v_scale,
+                         int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                         int32_t num_blocks)
+{
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        num_blocks < 0 || !k_scale || !v_scale)
+        return PGDO_EINVAL;
+    for (int32_t t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= (int64_t)num_blocks * block_size) return PGDO_EINVAL;
+        int64_t blk = slot / block_size, off = slot % block_size;
+        for (int32_t h = 0; h < num_kv_heads; ++h) {
+            int64_t src = ((int64_t)t * num_kv_heads + h) * head_dim;
+            int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * head_dim;
+            for (int32_t d = 0; d < head_dim; ++d) {
+                float kx = (float)pgdo_bf16_to_double(k_new[src + d]);
+                float vx = (float)pgdo_bf16_to_double(v_new[src + d]);
+                float ky = kx / k_scale[h];
+                float vy = vx / v_scale[h];
+                k_cache[dst + d] = pgdo_e4m3_from_double((double)ky);
+                v_cache[dst + d] = pgdo_e4m3_from_double((double)vy);
+            }
         }
     }
     return PGDO_OK;

@@ -10,6 +10,7 @@ import pytest
 import oracle
 from oracle import oracle as ormod
 import tests.test_oracle as pins
+import tests.test_oracle_quant as qpins
 
 SRC = os.path.join(os.path.dirname(ormod.__file__), "pgd_oracle.c")
 
@@ -38,6 +39,12 @@ MUTANTS = [
     ("dot product drops last dim", "for (int32_t d = 0; d < D; ++d) acc += qrow[d] * krow[d];",
      "for (int32_t d = 0; d + 1 < D; ++d) acc += qrow[d] * krow[d];", 0),
     ("q row of wrong head", "+ i) * a->head_dim;", "+ i / 2) * a->head_dim;", 0),
+    ("e4m3 ties away from zero", "nearbyint((ldexp(a, -E) - 1.0) * 8.0)",
+     "round((ldexp(a, -E) - 1.0) * 8.0)", 0),
+    ("e4m3 subnormal ties away", "nearbyint(ldexp(a, 9))", "round(ldexp(a, 9))", 0),
+    ("e4m3 NaN instead of saturation", "if (a >= 448.0) return (uint8_t)(sign | 0x7E);",
+     "if (a >= 448.0) return 0x7F;", 0),
+    ("quant K with V scale", "float ky = kx / k_scale[h];", "float ky = kx / v_scale[h];", 0),
 ]
 
 PIN_CALLS = [
@@ -55,6 +62,10 @@ PIN_CALLS = [
     ("tiled exact", lambda: pins.test_tiled_online_softmax_is_exact(None, 7, 13)),
     ("merge closed forms", lambda: pins.test_merge_partials_closed_forms(None)),
     ("kv append", lambda: pins.test_kv_append_is_a_byte_copy(None, __import__("numpy").uint16)),
+    ("e4m3 round trip", lambda: qpins.test_every_finite_code_round_trips(None)),
+    ("e4m3 midpoints", lambda: qpins.test_midpoints_round_to_even_mantissa(None)),
+    ("e4m3 saturation", lambda: qpins.test_saturation_and_special_values(None)),
+    ("quant append", lambda: qpins.test_kv_append_quant_divides_in_fp32_then_rounds(None)),
 ]
 
 
