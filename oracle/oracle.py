@@ -58,6 +58,8 @@ def configure(lib):
     args = [P, P, P, i32, P, P, P, i32, P, i32, i32, i32, i32, i32, i32, dbl]
     lib.pgdo_paged_decode.restype = ctypes.c_int
     lib.pgdo_paged_decode.argtypes = args + [P, P]
+    lib.pgdo_paged_decode_window.restype = ctypes.c_int
+    lib.pgdo_paged_decode_window.argtypes = args + [i32, P, P]
     lib.pgdo_paged_decode_rows.restype = ctypes.c_int
     lib.pgdo_paged_decode_rows.argtypes = args + [P, P, i32, P, P]
     lib.pgdo_paged_decode_tiled.restype = ctypes.c_int
@@ -231,3 +233,18 @@ def kv_append_quant(k_new, v_new, slot_mapping, k_cache, v_cache, k_scale, v_sca
     if rc:
         raise OracleError(f"pgdo_kv_append_quant rc={rc}")
     return k_cache, v_cache
+
+
+def paged_decode_window(q, k_cache, v_cache, block_table, context_lens, num_kv_heads, scale,
+                        window, k_scale=None, v_scale=None):
+    """Plain definition restricted to each sequence's last `window` tokens
+    (0 = full context)."""
+    args, keep, (B, Hq, D) = _decode_args(q, k_cache, v_cache, block_table, context_lens,
+                                          num_kv_heads, scale, k_scale, v_scale)
+    out = np.empty((B, Hq, D), np.float64)
+    lse = np.empty((B, Hq), np.float64)
+    rc = _load().pgdo_paged_decode_window(*args, int(window), _ptr(out), _ptr(lse))
+    if rc:
+        raise OracleError(f"pgdo_paged_decode_window rc={rc}")
+    del keep
+    return out, lse

@@ -213,6 +213,7 @@ typedef struct {
     const int32_t *context_lens;
     int32_t num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks;
     double scale;
+    int32_t window;             /* > 0: attend to the last `window` tokens only */
 } pgdo_args;
 
 static int check_args(const pgdo_args *a)
@@ -276,6 +277,9 @@ static double score(const double *qrow, const double *krow, int32_t D, double sc
 /* The plain definition, one (sequence, query head) row at a time.           */
 /* [P4-std]: S = Q K^T, P = softmax(S), O = P V, for a single query row.     */
 /* [P4-dec] / [P2-2.4]: query head i reads KV head i / g.                    */
+/* With a window W > 0 (sliding-window attention: the co-design page's       */
+/* principle 3 and "batching and attention" 2.3 name it as a way to cut the  */
+/* KV state read), the query at position n-1 sees tokens n-W .. n-1 only.    */
 /* ------------------------------------------------------------------------- */
 static void plain_row(const pgdo_args *a, int32_t s, int32_t i, double *out, double *lse)
 {
@@ -291,20 +295,21 @@ static void plain_row(const pgdo_args *a, int32_t s, int32_t i, double *out, dou
     double *qrow = malloc(sizeof(double) * D);
     double *row = malloc(sizeof(double) * D);
     double *x = malloc(sizeof(double) * n);
+    const int32_t lo = (a->window > 0 && n > a->window) ? n - a->window : 0;
     load_q(a, s, i, qrow);
     /* 1. all scores of the row */
-    for (int32_t t = 0; t < n; ++t) {
+    for (int32_t t = lo; t < n; ++t) {
         gather_row(a, a->k_cache, a->k_scale, s, h, t, row);
         x[t] = score(qrow, row, D, a->scale);
     }
     /* 2. softmax over the whole row: max, exponentials, sum */
-    double M = x[0];
-    for (int32_t t = 1; t < n; ++t) if (x[t] > M) M = x[t];
+    double M = x[lo];
+    for (int32_t t = lo + 1; t < n; ++t) if (x[t] > M) M = x[t];
     double Z = 0.0;
-    for (int32_t t = 0; t < n; ++t) { x[t] = exp(x[t] - M); Z += x[t]; }
+    for (int32_t t = lo; t < n; ++t) { x[t] = exp(x[t] - M); Z += x[t]; }
     /* 3. O = P V */
     for (int32_t d = 0; d < D; ++d) out[d] = 0.0;
-    for (int32_t t = 0; t < n; ++t) {
+    for (int32_t t = lo; t < n; ++t) {
         gather_row(a, a->v_cache, a->v_scale, s, h, t, row);
         for (int32_t d = 0; d < D; ++d) out[d] += x[t] * row[d];
     }
@@ -316,7 +321,7 @@ static void plain_row(const pgdo_args *a, int32_t s, int32_t i, double *out, dou
 #define ARGS_INIT                                                                \
     pgdo_args a = {q, k_cache, v_cache, kv_dtype, k_scale, v_scale, block_table, \
                    max_blocks_per_seq, context_lens, num_seqs, num_q_heads,      \
-                   num_kv_heads, head_dim, block_size, num_blocks, scale}
+                   num_kv_heads, head_dim, block_size, num_blocks, scale, 0}
 
 #define ARGS_DECL                                                                     \
     const uint16_t *q, const void *k_cache, const void *v_cache, int32_t kv_dtype,    \
@@ -332,6 +337,23 @@ int pgdo_paged_decode(ARGS_DECL, double *out, double *lse)
     ARGS_INIT;
     int rc = check_args(&a);
     if (rc) return rc;
+    for (int32_t s = 0; s < num_seqs; ++s)
+        for (int32_t i = 0; i < num_q_heads; ++i) {
+            int64_t r = (int64_t)s * num_q_heads + i;
+            plain_row(&a, s, i, out + r * head_dim, lse + r);
+        }
+    return PGDO_OK;
+}
+
+/* Whole batch with a sliding window of `window` tokens (0 = the full
+ * context): query row of sequence s sees tokens max(0, n-W) .. n-1. */
+int pgdo_paged_decode_window(ARGS_DECL, int32_t window, double *out, double *lse)
+{
+    ARGS_INIT;
+    int rc = check_args(&a);
+    if (rc) return rc;
+    if (window < 0) return PGDO_EINVAL;
+    a.window = window;
     for (int32_t s = 0; s < num_seqs; ++s)
         for (int32_t i = 0; i < num_q_heads; ++i) {
             int64_t r = (int64_t)s * num_q_heads + i;

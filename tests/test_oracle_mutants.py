@@ -11,6 +11,7 @@ import oracle
 from oracle import oracle as ormod
 import tests.test_oracle as pins
 import tests.test_oracle_quant as qpins
+import tests.test_oracle_window as wpins
 
 SRC = os.path.join(os.path.dirname(ormod.__file__), "pgd_oracle.c")
 
@@ -45,6 +46,8 @@ MUTANTS = [
     ("e4m3 NaN instead of saturation", "if (a >= 448.0) return (uint8_t)(sign | 0x7E);",
      "if (a >= 448.0) return 0x7F;", 0),
     ("quant K with V scale", "float ky = kx / k_scale[h];", "float ky = kx / v_scale[h];", 0),
+    ("window one token short", "? n - a->window : 0;", "? n - a->window + 1 : 0;", 0),
+    ("window ignored", "    a.window = window;\n", "", 0),
 ]
 
 PIN_CALLS = [
@@ -66,6 +69,8 @@ PIN_CALLS = [
     ("e4m3 midpoints", lambda: qpins.test_midpoints_round_to_even_mantissa(None)),
     ("e4m3 saturation", lambda: qpins.test_saturation_and_special_values(None)),
     ("quant append", lambda: qpins.test_kv_append_quant_divides_in_fp32_then_rounds(None)),
+    ("window of one", lambda: wpins.test_window_of_one_returns_last_value(None)),
+    ("window sdpa", lambda: wpins.test_window_matches_sdpa_on_last_tokens(None, 17)),
 ]
 
 
