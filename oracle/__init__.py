@@ -8,4 +8,5 @@ from .oracle import (  # noqa: F401
     BF16, E4M3, build_oracle, lib_path, bf16_to_double, e4m3_to_double,
     kv_append, paged_decode, paged_decode_rows, paged_decode_tiled,
     merge_partials, OracleError, e4m3_from_double, kv_append_quant, paged_decode_window,
+    paged_decode_multi,
 )

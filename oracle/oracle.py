@@ -58,6 +58,8 @@ def configure(lib):
     args = [P, P, P, i32, P, P, P, i32, P, i32, i32, i32, i32, i32, i32, dbl]
     lib.pgdo_paged_decode.restype = ctypes.c_int
     lib.pgdo_paged_decode.argtypes = args + [P, P]
+    lib.pgdo_paged_decode_multi.restype = ctypes.c_int
+    lib.pgdo_paged_decode_multi.argtypes = args + [i32, i32, P, P]
     lib.pgdo_paged_decode_window.restype = ctypes.c_int
     lib.pgdo_paged_decode_window.argtypes = args + [i32, P, P]
     lib.pgdo_paged_decode_rows.restype = ctypes.c_int
@@ -246,5 +248,23 @@ def paged_decode_window(q, k_cache, v_cache, block_table, context_lens, num_kv_h
     rc = _load().pgdo_paged_decode_window(*args, int(window), _ptr(out), _ptr(lse))
     if rc:
         raise OracleError(f"pgdo_paged_decode_window rc={rc}")
+    del keep
+    return out, lse
+
+
+def paged_decode_multi(q, k_cache, v_cache, block_table, context_lens, num_kv_heads, scale,
+                       window=0, k_scale=None, v_scale=None):
+    """Several query tokens per sequence: q [B][L][Hq][D] (uint16 bf16 bits);
+    returns out [B][L][Hq][D], lse [B][L][Hq]."""
+    q = _c(q, np.uint16)
+    B, L, Hq, D = q.shape
+    args, keep, _ = _decode_args(q.reshape(B, L * Hq, D), k_cache, v_cache, block_table,
+                                 context_lens, num_kv_heads, scale, k_scale, v_scale)
+    args[10] = Hq                    # num_q_heads (the flattened view used L * Hq)
+    out = np.empty((B, L, Hq, D), np.float64)
+    lse = np.empty((B, L, Hq), np.float64)
+    rc = _load().pgdo_paged_decode_multi(*args, int(L), int(window), _ptr(out), _ptr(lse))
+    if rc:
+        raise OracleError(f"pgdo_paged_decode_multi rc={rc}")
     del keep
     return out, lse

@@ -281,13 +281,13 @@ static double score(const double *qrow, const double *krow, int32_t D, double sc
 /* principle 3 and "batching and attention" 2.3 name it as a way to cut the  */
 /* KV state read), the query at position n-1 sees tokens n-W .. n-1 only.    */
 /* ------------------------------------------------------------------------- */
-static void plain_row(const pgdo_args *a, int32_t s, int32_t i, double *out, double *lse)
+/* One query row q (bf16) of sequence s against KV head h over tokens
+ * lo .. n-1; an empty range gives out = 0, lse = -inf. */
+static void attend(const pgdo_args *a, int32_t s, int32_t h, const uint16_t *q, int32_t lo,
+                   int32_t n, double *out, double *lse)
 {
     const int32_t D = a->head_dim;
-    const int32_t g = a->num_q_heads / a->num_kv_heads;
-    const int32_t h = i / g;
-    const int32_t n = a->context_lens[s];
-    if (n == 0) {
+    if (n <= lo) {
         for (int32_t d = 0; d < D; ++d) out[d] = 0.0;
         *lse = -INFINITY;
         return;
@@ -295,8 +295,7 @@ static void plain_row(const pgdo_args *a, int32_t s, int32_t i, double *out, dou
     double *qrow = malloc(sizeof(double) * D);
     double *row = malloc(sizeof(double) * D);
     double *x = malloc(sizeof(double) * n);
-    const int32_t lo = (a->window > 0 && n > a->window) ? n - a->window : 0;
-    load_q(a, s, i, qrow);
+    for (int32_t d = 0; d < D; ++d) qrow[d] = pgdo_bf16_to_double(q[d]);
     /* 1. all scores of the row */
     for (int32_t t = lo; t < n; ++t) {
         gather_row(a, a->k_cache, a->k_scale, s, h, t, row);
@@ -316,6 +315,15 @@ static void plain_row(const pgdo_args *a, int32_t s, int32_t i, double *out, dou
     for (int32_t d = 0; d < D; ++d) out[d] /= Z;
     *lse = M + log(Z);
     free(qrow); free(row); free(x);
+}
+
+static void plain_row(const pgdo_args *a, int32_t s, int32_t i, double *out, double *lse)
+{
+    const int32_t g = a->num_q_heads / a->num_kv_heads;
+    const int32_t h = i / g;
+    const int32_t n = a->context_lens[s];
+    const int32_t lo = (a->window > 0 && n > a->window) ? n - a->window : 0;
+    attend(a, s, h, a->q + ((int64_t)s * a->num_q_heads + i) * a->head_dim, lo, n, out, lse);
 }
 
 #define ARGS_INIT                                                                \
@@ -342,6 +350,33 @@ int pgdo_paged_decode(ARGS_DECL, double *out, double *lse)
             int64_t r = (int64_t)s * num_q_heads + i;
             plain_row(&a, s, i, out + r * head_dim, lse + r);
         }
+    return PGDO_OK;
+}
+
+/* Several query tokens per sequence (speculative-decoding verification, the
+ * lecture's section on it; prefill chunks that read a long prefix, the
+ * co-design page's agent section): q [num_seqs][q_len][num_q_heads][D]; the
+ * q_len newest tokens of sequence s sit at positions n-q_len .. n-1 (n =
+ * context_lens[s], which counts them), so query token i sees tokens below
+ * n - q_len + 1 + i (causal), and with window W > 0 only the last W of those.
+ * out [num_seqs][q_len][num_q_heads][D], lse [num_seqs][q_len][num_q_heads]. */
+int pgdo_paged_decode_multi(ARGS_DECL, int32_t q_len, int32_t window, double *out,
+                            double *lse)
+{
+    ARGS_INIT;
+    if (q_len < 1 || window < 0) return PGDO_EINVAL;
+    int rc = check_args(&a);
+    if (rc) return rc;
+    const int32_t g = num_q_heads / num_kv_heads;
+    for (int32_t s = 0; s < num_seqs; ++s)
+        for (int32_t it = 0; it < q_len; ++it)
+            for (int32_t i = 0; i < num_q_heads; ++i) {
+                const int64_t r = ((int64_t)s * q_len + it) * num_q_heads + i;
+                int32_t hi = context_lens[s] - q_len + 1 + it;
+                if (hi < 0) hi = 0;
+                const int32_t lo = (window > 0 && hi > window) ? hi - window : 0;
+                attend(&a, s, i / g, q + r * head_dim, lo, hi, out + r * head_dim, lse + r);
+            }
     return PGDO_OK;
 }
 

@@ -12,6 +12,7 @@ from oracle import oracle as ormod
 import tests.test_oracle as pins
 import tests.test_oracle_quant as qpins
 import tests.test_oracle_window as wpins
+import tests.test_oracle_multi as mpins
 
 SRC = os.path.join(os.path.dirname(ormod.__file__), "pgd_oracle.c")
 
@@ -48,6 +49,10 @@ MUTANTS = [
     ("quant K with V scale", "float ky = kx / k_scale[h];", "float ky = kx / v_scale[h];", 0),
     ("window one token short", "? n - a->window : 0;", "? n - a->window + 1 : 0;", 0),
     ("window ignored", "    a.window = window;\n", "", 0),
+    ("plain q row of wrong head", "+ i) * a->head_dim;", "+ i / 2) * a->head_dim;", 1),
+    ("causal limit one short", "context_lens[s] - q_len + 1 + it;", "context_lens[s] - q_len + it;", 0),
+    ("multi query token order", "((int64_t)s * q_len + it) * num_q_heads + i;",
+     "((int64_t)s * q_len + (q_len - 1 - it)) * num_q_heads + i;", 0),
 ]
 
 PIN_CALLS = [
@@ -71,6 +76,8 @@ PIN_CALLS = [
     ("quant append", lambda: qpins.test_kv_append_quant_divides_in_fp32_then_rounds(None)),
     ("window of one", lambda: wpins.test_window_of_one_returns_last_value(None)),
     ("window sdpa", lambda: wpins.test_window_matches_sdpa_on_last_tokens(None, 17)),
+    ("multi sdpa", lambda: mpins.test_matches_sdpa_with_causal_band_mask(None, 4, 0)),
+    ("multi window sdpa", lambda: mpins.test_matches_sdpa_with_causal_band_mask(None, 3, 5)),
 ]
 
 
