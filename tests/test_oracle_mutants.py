@@ -49,7 +49,7 @@ MUTANTS = [
     ("quant K with V scale", "float ky = kx / k_scale[h];", "float ky = kx / v_scale[h];", 0),
     ("window one token short", "? n - a->window : 0;", "? n - a->window + 1 : 0;", 0),
     ("window ignored", "    a.window = window;\n", "", 0),
-    ("plain q row of wrong head", "+ i) * a->head_dim;", "+ i / 2) * a->head_dim;", 1),
+    ("plain q row of wrong head", "+ i) * a->head_dim, lo, n", "+ i / 2) * a->head_dim, lo, n", 0),
     ("causal limit one short", "context_lens[s] - q_len + 1 + it;", "context_lens[s] - q_len + it;", 0),
     ("multi query token order", "((int64_t)s * q_len + it) * num_q_heads + i;",
      "((int64_t)s * q_len + (q_len - 1 - it)) * num_q_heads + i;", 0),
