@@ -104,6 +104,30 @@ pgd_status pgd_kv_append(const void *k_new, const void *v_new,
                          int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                          int32_t num_blocks, pgd_kv_dtype kv_dtype, void *stream);
 
+/*
+ * pgd_kv_append_quant -- the append of pgd_kv_append into an FP8 E4M3 cache
+ * from bf16 rows ("attention kernels", sections "paged KV and kernels" and
+ * "what to check": FP8 KV caches, read directly by the kernel).  Element x of
+ * KV head h is stored as the E4M3 value nearest to x / scale[h] (the division
+ * in fp32, IEEE round to nearest; the conversion rounds to nearest with ties
+ * to even and saturates magnitudes above 448 to +-448; NaN stays NaN), so
+ * that e4m3 * scale[h] approximates x.
+ *
+ *   k_new, v_new      device bf16 [num_tokens][num_kv_heads][head_dim],
+ *                     16-byte aligned
+ *   slot_mapping      device int64 [num_tokens], as pgd_kv_append
+ *   k_cache, v_cache  device E4M3 bytes, HND layout, 8-byte aligned
+ *   k_scale, v_scale  device fp32 [num_kv_heads] (the scales the decode uses)
+ *   head_dim in {128, 256}; block_size in {16, 32, 64}.
+ * Bit-exact with that definition.
+ */
+pgd_status pgd_kv_append_quant(const void *k_new, const void *v_new,
+                               const int64_t *slot_mapping, int32_t num_tokens,
+                               void *k_cache, void *v_cache,
+                               const float *k_scale, const float *v_scale,
+                               int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                               int32_t num_blocks, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* Paged decode attention                                                   */
 /* ------------------------------------------------------------------------ */

@@ -53,6 +53,8 @@ def load_library():
     lib.pgd_version.argtypes = []
     lib.pgd_kv_append.restype = st
     lib.pgd_kv_append.argtypes = [P, P, P, i32, P, P, i32, i32, i32, i32, st, P]
+    lib.pgd_kv_append_quant.restype = st
+    lib.pgd_kv_append_quant.argtypes = [P, P, P, i32, P, P, P, P, i32, i32, i32, i32, P]
     lib.pgd_decode_workspace_bytes.restype = sz
     lib.pgd_decode_workspace_bytes.argtypes = [i32, i32, i32, i32]
     lib.pgd_paged_decode_attention.restype = st
@@ -138,6 +140,28 @@ def kv_append(k_new, v_new, slot_mapping, k_cache, v_cache, *, stream=None) -> N
     _check(lib.pgd_kv_append(_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), k_new.shape[0],
                              _ptr(k_cache), _ptr(v_cache), hkv, d, bs, nb, _kv_dtype(k_cache),
                              _stream(stream)), "pgd_kv_append")
+
+
+def kv_append_quant(k_new, v_new, slot_mapping, k_cache, v_cache, k_scale, v_scale, *,
+                    stream=None) -> None:
+    """Quantise bf16 K/V rows of new tokens into an FP8 E4M3 cache
+    (pgd_kv_append_quant): byte = E4M3(x / scale[kv head])."""
+    lib = load_library()
+    _need(k_cache, "k_cache", (torch.uint8, torch.float8_e4m3fn), 4)
+    _need(v_cache, "v_cache", (k_cache.dtype,), 4)
+    _need(k_new, "k_new", (torch.bfloat16,), 3)
+    _need(v_new, "v_new", (torch.bfloat16,), 3)
+    _need(slot_mapping, "slot_mapping", (torch.int64,), 1)
+    _need(k_scale, "k_scale", (torch.float32,), 1)
+    _need(v_scale, "v_scale", (torch.float32,), 1)
+    nb, hkv, bs, d = k_cache.shape
+    if v_cache.shape != k_cache.shape or k_new.shape != v_new.shape or \
+            k_new.shape[1:] != (hkv, d) or slot_mapping.shape[0] != k_new.shape[0] or \
+            k_scale.shape != (hkv,) or v_scale.shape != (hkv,):
+        raise ValueError("kv_append_quant: inconsistent shapes")
+    _check(lib.pgd_kv_append_quant(_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), k_new.shape[0],
+                                   _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+                                   hkv, d, bs, nb, _stream(stream)), "pgd_kv_append_quant")
 
 
 def decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int,

@@ -222,6 +222,32 @@ pgd_status pgd_kv_append(const void *k_new, const void *v_new, const int64_t *sl
     return e == cudaSuccess ? PGD_OK : cuda_fail(e);
 }
 
+pgd_status pgd_kv_append_quant(const void *k_new, const void *v_new, const int64_t *slot_mapping,
+                               int32_t num_tokens, void *k_cache, void *v_cache,
+                               const float *k_scale, const float *v_scale, int32_t num_kv_heads,
+                               int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                               void *stream) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0) return PGD_ERR_INVALID_ARG;
+    if (head_dim != 128 && head_dim != 256) return PGD_ERR_UNSUPPORTED;
+    if (!supported_block(block_size)) return PGD_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PGD_OK;
+    if (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache || !k_scale || !v_scale)
+        return PGD_ERR_INVALID_ARG;
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 8) ||
+        !aligned(v_cache, 8) || !aligned(slot_mapping, 8) || !aligned(k_scale, 4) ||
+        !aligned(v_scale, 4))
+        return PGD_ERR_INVALID_ARG;
+    DeviceState *d = nullptr;
+    pgd_status st = device_state(&d);
+    if (st != PGD_OK) return st;
+    cudaError_t e = launch_kv_append_quant(k_new, v_new, slot_mapping, num_tokens, k_cache,
+                                           v_cache, k_scale, v_scale, num_kv_heads, head_dim,
+                                           block_size,
+                                           static_cast<int64_t>(num_blocks) * block_size,
+                                           d->flags, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PGD_OK : cuda_fail(e);
+}
+
 size_t pgd_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
                                   int32_t head_dim) {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||

@@ -55,6 +55,12 @@ cudaError_t launch_kv_append(const void *k_new, const void *v_new, const int64_t
                              int32_t row_bytes, int32_t block_size, int64_t pool_slots,
                              uint32_t *flags, cudaStream_t stream);
 
+cudaError_t launch_kv_append_quant(const void *k_new, const void *v_new, const int64_t *slots,
+                                   int32_t num_tokens, void *k_cache, void *v_cache,
+                                   const float *k_scale, const float *v_scale, int32_t hkv,
+                                   int32_t head_dim, int32_t block_size, int64_t pool_slots,
+                                   uint32_t *flags, cudaStream_t stream);
+
 cudaError_t launch_merge_partials(const float *o_part, const float *lse_part, int32_t parts,
                                   int32_t rows, int32_t head_dim, uint16_t *out, float *lse_out,
                                   cudaStream_t stream);

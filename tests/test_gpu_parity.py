@@ -265,3 +265,55 @@ def test_fused_decode_step(ctx, Hq, Hkv, D, bs, dt, nctas):
     got = to_f64(out1)
     assert np.all(np.isfinite(got))
     assert_close(got, ref, dt, "fused step")
+
+
+# --------------------------------------------------------------------------- #
+# quantising append: bf16 rows -> E4M3 cache, bit-exact with the oracle
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("D,bs", [(128, 16), (256, 32), (128, 64)])
+def test_kv_append_quant_bit_exact(D, bs):
+    from workloads import to_bf16_bits
+    rng = np.random.default_rng(300 + D + bs)
+    N, Hkv, nb = 57, 4, 40
+    x = rng.standard_normal((2, N, Hkv, D)).astype(np.float32) * 3
+    x[:, :5] *= 1e3                      # saturate
+    x[:, 5:10] *= 1e-4                   # subnormal codes
+    x[:, 10, :, :4] = [1.0625, 1.1875, -3.25, 0.0]   # exact midpoints at scale 1
+    kb, vb = to_bf16_bits(x[0]), to_bf16_bits(x[1])
+    ks = np.array([1.0, 0.0071, 0.02, 0.5], np.float32)
+    vs = np.array([0.003, 1.0, 0.25, 2.0], np.float32)
+    slots = rng.choice(nb * bs, size=N, replace=False).astype(np.int64)
+    slots[3] = -1
+    kc0 = rng.integers(0, 256, size=(nb, Hkv, bs, D)).astype(np.uint8)
+    vc0 = rng.integers(0, 256, size=(nb, Hkv, bs, D)).astype(np.uint8)
+    ek, ev = oracle.kv_append_quant(kb, vb, slots, kc0, vc0, ks, vs, bs)
+    from tests.gpu_helpers import dev_bf16
+    kc = torch.from_numpy(kc0.copy()).cuda()
+    vc = torch.from_numpy(vc0.copy()).cuda()
+    pgd.kv_append_quant(dev_bf16(kb), dev_bf16(vb), torch.from_numpy(slots).cuda(), kc, vc,
+                        torch.from_numpy(ks).cuda(), torch.from_numpy(vs).cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(kc.cpu().numpy(), ek) and np.array_equal(vc.cpu().numpy(), ev)
+
+
+def test_quantised_append_then_fp8_decode():
+    """bf16 K/V quantised by the library, then decoded from the FP8 cache."""
+    from tests.gpu_helpers import dev_bf16
+    from workloads import to_bf16_bits
+    w = make_case([70, 300, 16, 1], 32, 4, 128, 16, "e4m3", seed=310)
+    rng = np.random.default_rng(311)
+    live = [s for s in range(w.num_seqs) if w.context_lens[s] > 0]
+    slots = np.array([int(w.block_table[s, (w.context_lens[s] - 1) // 16]) * 16 +
+                      int((w.context_lens[s] - 1) % 16) for s in live], np.int64)
+    kb = to_bf16_bits(rng.standard_normal((len(slots), 4, 128)).astype(np.float32))
+    vb = to_bf16_bits(rng.standard_normal((len(slots), 4, 128)).astype(np.float32))
+    ek, ev = oracle.kv_append_quant(kb, vb, slots, w.k_cache, w.v_cache, w.k_scale, w.v_scale, 16)
+    d = Dev(w)
+    pgd.kv_append_quant(dev_bf16(kb), dev_bf16(vb), torch.from_numpy(slots).cuda(), d.k, d.v,
+                        d.ks, d.vs)
+    out, _ = d.decode()
+    torch.cuda.synchronize()
+    assert np.array_equal(d.k.cpu().numpy(), ek) and np.array_equal(d.v.cpu().numpy(), ev)
+    w.k_cache, w.v_cache = ek, ev
+    ref, _ = oracle_full(w)
+    assert_close(to_f64(out), ref, "e4m3", "quantised append + decode")
