@@ -172,8 +172,8 @@ size_t pgd_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
  *   max_context_len  host hint >= every context length (0 = unknown); only
  *                 used to size the grid for small batches
  *   num_q_heads % num_kv_heads == 0, g = num_q_heads / num_kv_heads in
- *                 {1, 2, 4, 8, 16}; head_dim in {128, 256} (256 with bf16
- *                 only); block_size in {16, 32, 64}
+ *                 1 .. 16; head_dim in {128, 256} (256 with bf16 only);
+ *                 block_size in {16, 32, 64}
  *   scale         softmax scale applied to q.k (e.g. 1/sqrt(head_dim))
  *   kv_dtype      PGD_KV_BF16 or PGD_KV_FP8_E4M3
  *   k_scale, v_scale  device fp32 [num_kv_heads] for FP8 (NULL for bf16)
@@ -224,6 +224,43 @@ pgd_status pgd_decode_step(
     const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
     const int32_t *block_table, int32_t max_blocks_per_seq,
     const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t num_blocks, float scale, pgd_kv_dtype kv_dtype,
+    const float *k_scale, const float *v_scale,
+    void *out, float *lse_out,
+    void *workspace, size_t workspace_bytes, int32_t num_ctas, void *stream);
+
+/*
+ * pgd_paged_decode_attention_ex -- pgd_paged_decode_attention generalised to
+ * q_len query tokens per sequence and an optional sliding window.
+ *
+ * The q_len newest tokens of sequence s occupy positions n - q_len .. n - 1
+ * (n = context_lens[s] counts them, their K/V already in the cache).  Query
+ * token j (0 <= j < q_len) sees positions t < hi = n - q_len + 1 + j (causal
+ * among the new tokens, as in the verification step of speculative decoding
+ * in the inference lecture's section on it), and with window > 0 only
+ * t >= hi - window (sliding-window attention, the co-design page's section on
+ * reducing the attended range).  A row that sees no position gets out = 0 and
+ * lse = -inf; the formulas are otherwise those of
+ * pgd_paged_decode_attention over the visible positions.
+ *
+ *   q        device bf16 [num_seqs][q_len][num_q_heads][head_dim]
+ *   out      device bf16 [num_seqs][q_len][num_q_heads][head_dim]
+ *   lse_out  optional fp32 [num_seqs][q_len][num_q_heads]
+ *   q_len    >= 1 with g * q_len <= 16 (g = num_q_heads / num_kv_heads): every
+ *            query row of a KV head rides on one pass over its K/V tiles
+ *   window   0 = the whole causal range; > 0 = the last `window` positions
+ *   workspace  at least pgd_decode_workspace_bytes(num_seqs,
+ *            num_q_heads * q_len, num_kv_heads, head_dim) bytes, or NULL/0
+ *   all other arguments and errors as pgd_paged_decode_attention; q_len = 1,
+ *   window = 0 gives exactly that call.  g * q_len > 16 returns
+ *   PGD_ERR_UNSUPPORTED.  Blocks that lie wholly before a window are not read.
+ */
+pgd_status pgd_paged_decode_attention_ex(
+    const void *q, const void *k_cache, const void *v_cache,
+    const int32_t *block_table, int32_t max_blocks_per_seq,
+    const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
+    int32_t q_len, int32_t window,
     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
     int32_t num_blocks, float scale, pgd_kv_dtype kv_dtype,
     const float *k_scale, const float *v_scale,

@@ -5,12 +5,12 @@ this package only marshals torch tensors to it.
 """
 from ._binding import (  # noqa: F401
     PGD_KV_BF16, PGD_KV_FP8_E4M3, PGDError, LIB_PATH, lib_path, load_library, kv_append,
-    kv_append_quant,
-    paged_decode_attention, paged_decode_attention_noalloc, decode_step, merge_partials, decode_workspace_bytes,
+    kv_append_quant, paged_decode_attention, paged_decode_attention_ex,
+    paged_decode_attention_noalloc, decode_step, merge_partials, decode_workspace_bytes,
     get_device_error, shutdown,
 )
 
-__all__ = ["kv_append", "kv_append_quant", "paged_decode_attention", "paged_decode_attention_noalloc", "decode_step",
-           "merge_partials", "decode_workspace_bytes",
-           "get_device_error", "shutdown", "PGDError", "load_library",
+__all__ = ["kv_append", "kv_append_quant", "paged_decode_attention", "paged_decode_attention_ex",
+           "paged_decode_attention_noalloc", "decode_step", "merge_partials",
+           "decode_workspace_bytes", "get_device_error", "shutdown", "PGDError", "load_library",
            "lib_path", "PGD_KV_BF16", "PGD_KV_FP8_E4M3"]

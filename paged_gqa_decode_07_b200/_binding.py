@@ -60,6 +60,10 @@ def load_library():
     lib.pgd_paged_decode_attention.restype = st
     lib.pgd_paged_decode_attention.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32, i32,
                                                i32, f32, st, P, P, P, P, P, sz, i32, P]
+    lib.pgd_paged_decode_attention_ex.restype = st
+    lib.pgd_paged_decode_attention_ex.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32,
+                                                  i32, i32, i32, i32, f32, st, P, P, P, P, P, sz,
+                                                  i32, P]
     lib.pgd_decode_step.restype = st
     lib.pgd_decode_step.argtypes = [P, P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, i32, i32,
                                     f32, st, P, P, P, P, P, sz, i32, P]
@@ -212,6 +216,53 @@ def paged_decode_attention(q, k_cache, v_cache, block_table, context_lens, num_q
         block_size, k_cache.shape[0], float(scale), kvd, _ptr(k_scale), _ptr(v_scale), _ptr(out),
         _ptr(lse_out), _ptr(workspace), ws_bytes, int(num_ctas), _stream(stream)),
         "pgd_paged_decode_attention")
+    return out
+
+
+def paged_decode_attention_ex(q, k_cache, v_cache, block_table, context_lens, num_q_heads: int,
+                              num_kv_heads: int, head_dim: int, block_size: int, scale: float,
+                              out: Optional[torch.Tensor] = None, *, window: int = 0,
+                              max_context_len: int = 0, k_scale=None, v_scale=None, lse_out=None,
+                              workspace=None, num_ctas: int = 0, stream=None) -> torch.Tensor:
+    """Decode attention for q_len query tokens per sequence with an optional
+    sliding window (pgd_paged_decode_attention_ex).
+
+    q bf16 [B][q_len][Hq][D]: the q_len newest tokens of each sequence, already
+    counted in context_lens; token j sees positions below
+    context_lens - q_len + 1 + j, and with window > 0 only the last `window` of
+    them.  Returns out (bf16 [B][q_len][Hq][D]); lse_out (fp32 [B][q_len][Hq])
+    is filled when given.  Other arguments as paged_decode_attention.
+    """
+    lib = load_library()
+    _need(q, "q", (torch.bfloat16,), 4)
+    _need(k_cache, "k_cache", _KV_DTYPES, 4)
+    _need(v_cache, "v_cache", (k_cache.dtype,), 4)
+    _need(block_table, "block_table", (torch.int32,), 2)
+    _need(context_lens, "context_lens", (torch.int32,), 1)
+    B, L = q.shape[0], q.shape[1]
+    if q.shape != (B, L, num_q_heads, head_dim) or tuple(k_cache.shape[1:]) != (
+            num_kv_heads, block_size, head_dim) or v_cache.shape != k_cache.shape or \
+            block_table.shape[0] != B or context_lens.shape[0] != B:
+        raise ValueError("paged_decode_attention_ex: inconsistent shapes")
+    kvd = _kv_dtype(k_cache)
+    if kvd == PGD_KV_FP8_E4M3:
+        _need(k_scale, "k_scale", (torch.float32,), 1)
+        _need(v_scale, "v_scale", (torch.float32,), 1)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", (torch.bfloat16,), 4)
+    if lse_out is not None:
+        _need(lse_out, "lse_out", (torch.float32,), 3)
+    ws_bytes = 0
+    if workspace is not None:
+        _need(workspace, "workspace", None)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.pgd_paged_decode_attention_ex(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), block_table.shape[1],
+        _ptr(context_lens), B, int(max_context_len), L, int(window), num_q_heads, num_kv_heads,
+        head_dim, block_size, k_cache.shape[0], float(scale), kvd, _ptr(k_scale), _ptr(v_scale),
+        _ptr(out), _ptr(lse_out), _ptr(workspace), ws_bytes, int(num_ctas), _stream(stream)),
+        "pgd_paged_decode_attention_ex")
     return out
 
 

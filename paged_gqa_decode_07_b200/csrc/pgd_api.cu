@@ -166,7 +166,7 @@ bool pick_variant(int D, int bs, int nt, bool fp8, Variant *v) {
 }
 
 bool supported_block(int bs) { return bs == 16 || bs == 32 || bs == 64; }
-bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
+bool supported_group(int g) { return g >= 1 && g <= 16; }
 
 // Fixed cost of one (sequence, KV head) unit in a CTA (descriptor, query
 // rows, block-table fetch, first-tile latency, output) expressed as the K/V
@@ -273,10 +273,11 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
                        pgd_kv_dtype kv_dtype, const float *k_scale, const float *v_scale,
                        const void *k_new, const void *v_new, void *out, float *lse_out,
                        void *workspace, size_t workspace_bytes, int32_t num_ctas,
-                       void *stream) {
+                       void *stream, int32_t q_len = 1, int32_t window = 0) {
     // ---- host-side checks (nothing is enqueued on failure) ------------------
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
-        max_blocks_per_seq <= 0 || max_context_len < 0 || num_ctas < 0)
+        max_blocks_per_seq <= 0 || max_context_len < 0 || num_ctas < 0 || q_len < 1 ||
+        window < 0)
         return PGD_ERR_INVALID_ARG;
     if (num_q_heads % num_kv_heads) return PGD_ERR_INVALID_ARG;
     if (kv_dtype != PGD_KV_BF16 && kv_dtype != PGD_KV_FP8_E4M3) return PGD_ERR_INVALID_ARG;
@@ -286,6 +287,8 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     if (!supported_group(g) || !supported_block(block_size)) return PGD_ERR_UNSUPPORTED;
     if (head_dim != 128 && head_dim != 256) return PGD_ERR_UNSUPPORTED;
     if (fp8 && head_dim != 128) return PGD_ERR_UNSUPPORTED;
+    const int rows = g * q_len;                 // query rows per (sequence, KV head)
+    if (rows > 16) return PGD_ERR_UNSUPPORTED;
     if (static_cast<long long>(num_blocks) * num_kv_heads >= INT_MAX ||
         static_cast<long long>(max_blocks_per_seq) * block_size >= INT_MAX)
         return PGD_ERR_UNSUPPORTED;
@@ -300,11 +303,12 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     if (!workspace && workspace_bytes) return PGD_ERR_INVALID_ARG;
     if ((k_new == nullptr) != (v_new == nullptr)) return PGD_ERR_INVALID_ARG;
     if (k_new && (!aligned(k_new, 16) || !aligned(v_new, 16))) return PGD_ERR_INVALID_ARG;
+    if (k_new && q_len != 1) return PGD_ERR_UNSUPPORTED;   // fused append: one new token
 
     DeviceState *d = nullptr;
     pgd_status st = device_state(&d);
     if (st != PGD_OK) return st;
-    const int nt = g > 8 ? 2 : 1;
+    const int nt = rows > 8 ? 2 : 1;
     Variant var;
     if (!pick_variant(head_dim, block_size, nt, fp8, &var)) return PGD_ERR_UNSUPPORTED;
 
@@ -325,7 +329,7 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     if (grid > (1LL << 24)) return PGD_ERR_INVALID_ARG;
 
     // ---- workspace --------------------------------------------------------------
-    const WsLayout lay = ws_layout(g, head_dim, grid);
+    const WsLayout lay = ws_layout(rows, head_dim, grid);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if ((st = ensure_counters(d, static_cast<long long>(num_seqs) * num_kv_heads, s)) != PGD_OK)
@@ -355,9 +359,9 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     DecodeLaunchArgs a;
     std::memset(&a, 0, sizeof(a));
     const int E = fp8 ? 1 : 2;
-    const long long rows = static_cast<long long>(num_blocks) * num_kv_heads;
-    if ((st = encode_kv_map(&a.tmK, k_cache, head_dim, E, block_size, rows)) != PGD_OK) return st;
-    if ((st = encode_kv_map(&a.tmV, v_cache, head_dim, E, block_size, rows)) != PGD_OK) return st;
+    const long long kv_rows = static_cast<long long>(num_blocks) * num_kv_heads;
+    if ((st = encode_kv_map(&a.tmK, k_cache, head_dim, E, block_size, kv_rows)) != PGD_OK) return st;
+    if ((st = encode_kv_map(&a.tmV, v_cache, head_dim, E, block_size, kv_rows)) != PGD_OK) return st;
     DecodeParams &p = a.p;
     p.q = static_cast<const uint16_t *>(q);
     p.out = static_cast<uint16_t *>(out);
@@ -382,6 +386,9 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     p.num_blocks = num_blocks;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.unit_cost = unit_cost_tiles(head_dim, block_size, fp8);
+    p.q_len = q_len;
+    p.window = window;
+    p.rows = rows;
     a.grid = static_cast<int>(grid);
     a.stream = s;
     cudaError_t e = var.launch(a);
@@ -417,6 +424,20 @@ pgd_status pgd_decode_step(
                        num_seqs, max_context_len, num_q_heads, num_kv_heads, head_dim,
                        block_size, num_blocks, scale, kv_dtype, k_scale, v_scale, k_new, v_new,
                        out, lse_out, workspace, workspace_bytes, num_ctas, stream);
+}
+
+pgd_status pgd_paged_decode_attention_ex(
+    const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+    int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
+    int32_t max_context_len, int32_t q_len, int32_t window, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
+    pgd_kv_dtype kv_dtype, const float *k_scale, const float *v_scale, void *out,
+    float *lse_out, void *workspace, size_t workspace_bytes, int32_t num_ctas, void *stream) {
+    return decode_impl(q, k_cache, v_cache, block_table, max_blocks_per_seq, context_lens,
+                       num_seqs, max_context_len, num_q_heads, num_kv_heads, head_dim,
+                       block_size, num_blocks, scale, kv_dtype, k_scale, v_scale, nullptr,
+                       nullptr, out, lse_out, workspace, workspace_bytes, num_ctas, stream,
+                       q_len, window);
 }
 
 pgd_status pgd_merge_partials(const float *o_part, const float *lse_part, int32_t num_parts,
@@ -640,6 +661,9 @@ extern "C" pgd_status pgd_paged_decode_attention_noalloc(
     p.num_blocks = num_blocks;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.unit_cost = unit_cost_tiles(head_dim, block_size, fp8);
+    p.q_len = 1;
+    p.window = 0;
+    p.rows = g;
     a.grid = static_cast<int>(grid);
     a.stream = s;
     e = var.launch(a);

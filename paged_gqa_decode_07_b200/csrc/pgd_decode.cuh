@@ -64,13 +64,18 @@ struct DecodeParams {
     uint8_t *k_cache;             // raw cache pointers (fused append only)
     uint8_t *v_cache;
     int32_t *counters;            // [B * Hkv], zero between calls
-    float *o_part;                // [2 * grid][g][D]
-    float *lse_part;              // [2 * grid][g], log2 domain
+    float *o_part;                // [2 * grid][rows][D]
+    float *lse_part;              // [2 * grid][rows], log2 domain
     uint32_t *flags;              // device flag word
     int32_t max_blocks_per_seq;
     int32_t num_seqs, num_q_heads, num_kv_heads, group, num_blocks;
     float scale_log2;             // softmax scale * log2(e)
     int32_t unit_cost;            // work weight of a unit's fixed cost, in tiles
+    // query rows per unit: q_len query tokens x group heads (rows <= 16).  q,
+    // out are [B][q_len][Hq][D], lse [B][q_len][Hq]; query token i of a
+    // sequence with n tokens sits at position n - q_len + i and sees tokens
+    // below n - q_len + 1 + i, and with window > 0 only the last window of them.
+    int32_t q_len, window, rows;
 };
 
 constexpr int kConsumerWarps = 4;
@@ -87,7 +92,7 @@ struct SegDesc {
     int s, h, j0, j1, n, ctx;
     int terminal;     // 1: no more segments for this CTA
     float ksc, vsc;   // FP8 per-KV-head scales (1 for bf16)
-    int pad;
+    int jlo;          // first block any query row of the unit sees
 };
 
 template <int D, int BS, int NT, bool FP8, int NSTAGES>
@@ -194,13 +199,29 @@ __device__ __forceinline__ long long unit_weight(int n, int unit_cost) {
     return n > 0 ? (long long)n + unit_cost : 0;
 }
 
+// First block any query row of a unit with ctx tokens sees: the window of
+// its first query token (position ctx - q_len) starts there; 0 without one.
+template <int BS>
+__device__ __forceinline__ int first_block(int ctx, const DecodeParams &p) {
+    if (p.window <= 0) return 0;
+    return max(0, ctx - p.q_len + 1 - p.window) / BS;
+}
+
 // Walk over the units of a CTA's work range (producer and appender).  Unit
-// (s, h) occupies work indices [a, a + w): its n tiles first, then the
-// fixed-cost slots, which hold no tiles.
+// (s, h) reads blocks jlo .. n-1 and occupies work indices [a, a + w): its
+// n - jlo tiles first, then the fixed-cost slots, which hold no tiles.
 struct Cursor {
-    int s, h, n, ctx;
+    int s, h, n, ctx, jlo;
     long long a, w;
 };
+
+template <int BS>
+__device__ __forceinline__ void set_seq(Cursor &c, const DecodeParams &p) {
+    c.ctx = ctx_of<BS>(p, c.s);
+    c.n = nblk_of<BS>(c.ctx);
+    c.jlo = first_block<BS>(c.ctx, p);
+    c.w = unit_weight(c.n - c.jlo, p.unit_cost);
+}
 
 template <int BS>
 __device__ __forceinline__ void next_unit(Cursor &c, const DecodeParams &p) {
@@ -208,11 +229,9 @@ __device__ __forceinline__ void next_unit(Cursor &c, const DecodeParams &p) {
     if (++c.h == p.num_kv_heads) {
         c.h = 0;
         for (++c.s; c.s < p.num_seqs; ++c.s) {
-            c.ctx = ctx_of<BS>(p, c.s);
-            c.n = nblk_of<BS>(c.ctx);
+            set_seq<BS>(c, p);
             if (c.n) break;
         }
-        c.w = unit_weight(c.n, p.unit_cost);
     }
 }
 
@@ -221,12 +240,18 @@ __device__ __forceinline__ Cursor first_unit(const DecodeParams &p, int s0, long
                                             long long u0) {
     Cursor c;
     c.s = s0;
-    c.ctx = ctx_of<BS>(p, s0);
-    c.n = nblk_of<BS>(c.ctx);
-    c.w = unit_weight(c.n, p.unit_cost);
+    set_seq<BS>(c, p);
     c.h = (int)((u0 - pfx0) / c.w);
     c.a = pfx0 + (long long)c.h * c.w;
     return c;
+}
+
+// Work weight of sequence s per KV head (prologue sums and the locate scan).
+template <int BS>
+__device__ __forceinline__ long long seq_weight(const DecodeParams &p, int s) {
+    const int ctx = ctx_of<BS>(p, s);
+    const int n = nblk_of<BS>(ctx);
+    return unit_weight(n - first_block<BS>(ctx, p), p.unit_cost);
 }
 
 __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uint32_t bytes,
@@ -257,11 +282,16 @@ __device__ __forceinline__ long long lds64(uint32_t a) {
 template <int D>
 __device__ __forceinline__ void merge_unit(const DecodeParams &p, long long ua, long long U,
                                            long long G, long long c_first, long long c_last,
-                                           long long row0, int g) {
+                                           int s, int h) {
     constexpr int V4 = D / 4;                      // float4 columns per row
-    constexpr int MAXC = (V4 + 7) / 8;             // columns per thread when g = 16
-    const int tph = kConsumers / g;                // threads per head (g <= 16)
-    const int head = threadIdx.x / tph, sub = threadIdx.x % tph;
+    constexpr int MAXC = (V4 + 7) / 8;             // columns per thread when rows = 16
+    const int R = p.rows, g = p.group;
+    const int tph = kConsumers / R;                // threads per query row (R <= 16)
+    const int head = threadIdx.x / tph, sub = threadIdx.x % tph;   // head: the query row
+    if (head >= R) return;                         // 128 / R need not be exact
+    // output row of query row `head`: query token head / g, head h*g + head % g
+    const long long orow =
+        ((long long)s * p.q_len + head / g) * p.num_q_heads + (long long)h * g + head % g;
     auto slot_of = [&](long long c) { return 2 * c + ((ua <= c * U / G) ? 0 : 1); };
     // pass 1: M over the pieces
     float M = -INFINITY;
@@ -269,11 +299,11 @@ __device__ __forceinline__ void merge_unit(const DecodeParams &p, long long ua, 
     for (; c + 3 <= c_last; c += 4) {
         float l[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) l[i] = __ldcg(p.lse_part + slot_of(c + i) * g + head);
+        for (int i = 0; i < 4; ++i) l[i] = __ldcg(p.lse_part + slot_of(c + i) * R + head);
 #pragma unroll
         for (int i = 0; i < 4; ++i) M = fmaxf(M, l[i]);
     }
-    for (; c <= c_last; ++c) M = fmaxf(M, __ldcg(p.lse_part + slot_of(c) * g + head));
+    for (; c <= c_last; ++c) M = fmaxf(M, __ldcg(p.lse_part + slot_of(c) * R + head));
     const float Mu = M == -INFINITY ? 0.f : M;
     // pass 2: weighted sum of the partial rows
     float4 acc[MAXC];
@@ -281,7 +311,7 @@ __device__ __forceinline__ void merge_unit(const DecodeParams &p, long long ua, 
     for (int i = 0; i < MAXC; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     float W = 0.f;
     auto add_piece = [&](long long cc, float w) {
-        const float4 *row = reinterpret_cast<const float4 *>(p.o_part + (slot_of(cc) * g + head) * D);
+        const float4 *row = reinterpret_cast<const float4 *>(p.o_part + (slot_of(cc) * R + head) * D);
 #pragma unroll
         for (int i = 0; i < MAXC; ++i) {
             const int col = sub + i * tph;
@@ -292,14 +322,14 @@ __device__ __forceinline__ void merge_unit(const DecodeParams &p, long long ua, 
         }
     };
     for (c = c_first; c + 1 <= c_last; c += 2) {
-        const float w0 = ex2(__ldcg(p.lse_part + slot_of(c) * g + head) - Mu);
-        const float w1 = ex2(__ldcg(p.lse_part + slot_of(c + 1) * g + head) - Mu);
+        const float w0 = ex2(__ldcg(p.lse_part + slot_of(c) * R + head) - Mu);
+        const float w1 = ex2(__ldcg(p.lse_part + slot_of(c + 1) * R + head) - Mu);
         W += w0 + w1;
         add_piece(c, w0);
         add_piece(c + 1, w1);
     }
     if (c <= c_last) {
-        const float w0 = ex2(__ldcg(p.lse_part + slot_of(c) * g + head) - Mu);
+        const float w0 = ex2(__ldcg(p.lse_part + slot_of(c) * R + head) - Mu);
         W += w0;
         add_piece(c, w0);
     }
@@ -311,11 +341,11 @@ __device__ __forceinline__ void merge_unit(const DecodeParams &p, long long ua, 
             uint2 packed;
             packed.x = pack_bf16x2(acc[i].x * inv, acc[i].y * inv);
             packed.y = pack_bf16x2(acc[i].z * inv, acc[i].w * inv);
-            *reinterpret_cast<uint2 *>(p.out + (row0 + head) * D + 4 * col) = packed;
+            *reinterpret_cast<uint2 *>(p.out + orow * D + 4 * col) = packed;
         }
     }
     if (p.lse_out && sub == 0)
-        p.lse_out[row0 + head] = W > 0.f ? (M + log2f(W)) * kLn2 : -INFINITY;
+        p.lse_out[orow] = W > 0.f ? (M + log2f(W)) * kLn2 : -INFINITY;
 }
 
 // ------------------------------------------------------------------ kernel
@@ -375,24 +405,26 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
 
     // ---- prologue: total tiles and this CTA's range --------------------
     long long mine = 0;
-    for (int s = tid; s < B; s += kThreads)
-        mine += unit_weight(nblk_of<BS>(ctx_of<BS>(p, s)), p.unit_cost);
+    for (int s = tid; s < B; s += kThreads) mine += seq_weight<BS>(p, s);
     const long long U = block_sum(mine, misc) * Hkv;
     // CTAs beyond the tile count get no range, so every range is non-empty
     const long long G = min((long long)gridDim.x, U);
     const long long u0 = cta < G ? cta * U / G : 0, u1 = cta < G ? (cta + 1) * U / G : 0;
 
-    // units with an empty context: out = 0, lse = -inf (each thread checks
-    // its own units, spread over all CTAs)
+    // units with an empty context: out = 0, lse = -inf for all their query
+    // rows (each thread checks its own units, spread over all CTAs)
     for (long long v = cta + (long long)gridDim.x * tid; v < (long long)B * Hkv;
          v += (long long)gridDim.x * kThreads) {
         const int s = (int)(v / Hkv), h = (int)(v % Hkv);
         if (ctx_of<BS>(p, s) != 0) continue;
-        const long long row0 = (long long)s * p.num_q_heads + (long long)h * g;
-        uint16_t *o = p.out + row0 * D;
-        for (int e = 0; e < g * D; ++e) o[e] = 0;
-        if (p.lse_out)
-            for (int e = 0; e < g; ++e) p.lse_out[row0 + e] = -INFINITY;
+        for (int i = 0; i < p.q_len; ++i) {
+            const long long row0 =
+                ((long long)s * p.q_len + i) * p.num_q_heads + (long long)h * g;
+            uint16_t *o = p.out + row0 * D;
+            for (int e = 0; e < g * D; ++e) o[e] = 0;
+            if (p.lse_out)
+                for (int e = 0; e < g; ++e) p.lse_out[row0 + e] = -INFINITY;
+        }
     }
     if (u0 >= u1) return;   // nothing in flight, no barrier shared past this point
 
@@ -401,8 +433,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         long long base = 0;
         for (int sb = 0; sb < B; sb += kThreads) {
             const int s = sb + tid;
-            const long long wgt =
-                s < B ? unit_weight(nblk_of<BS>(ctx_of<BS>(p, s)), p.unit_cost) * Hkv : 0;
+            const long long wgt = s < B ? seq_weight<BS>(p, s) * Hkv : 0;
             long long tot;
             const long long incl = block_scan(wgt, tot, misc);
             const long long excl = base + incl - wgt;
@@ -430,9 +461,9 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         Cursor cur = first_unit<BS>(p, misc->s0, misc->pfx0, u0);
         uint32_t ait = 0;
         for (; cur.a < u1; next_unit<BS>(cur, p)) {
-            const long long j0 = max(0LL, u0 - cur.a);
-            const int j1 = (int)min((long long)cur.n, u1 - cur.a);
-            if (j0 < j1 && j1 == cur.n) {
+            const long long r0 = max(0LL, u0 - cur.a);
+            const long long r1 = min((long long)(cur.n - cur.jlo), u1 - cur.a);
+            if (r0 < r1 && cur.jlo + r1 == cur.n) {
                 const uint32_t as = ait % kAppSlots;
                 bool ok = true;
                 if (lane == 0 && ait >= (uint32_t)kAppSlots)
@@ -470,13 +501,14 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
     if (warp == kConsumerWarps) {
         // ================= producer warp ====================================
         Cursor cur = first_unit<BS>(p, misc->s0, misc->pfx0, u0);
-        const uint32_t qbytes = (uint32_t)(g * D * 2);
+        const uint32_t qtok = (uint32_t)(g * D * 2);          // one query token's rows
         uint32_t it = 0, sit = 0, ait = 0;
         bool ok = true;
         for (; cur.a < u1 && ok; next_unit<BS>(cur, p)) {
-            const int j0 = (int)max(0LL, u0 - cur.a);
-            const int j1 = (int)min((long long)cur.n, u1 - cur.a);
-            if (j0 >= j1) continue;   // the range holds only this unit's fixed-cost slots
+            const int r0 = (int)max(0LL, u0 - cur.a);
+            const int r1 = (int)min((long long)(cur.n - cur.jlo), u1 - cur.a);
+            if (r0 >= r1) continue;   // the range holds only this unit's fixed-cost slots
+            const int j0 = cur.jlo + r0, j1 = cur.jlo + r1;   // absolute blocks
             // -- descriptor and query rows of the segment
             {
                 const uint32_t slot = sit % C::NSEG;
@@ -486,7 +518,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 if (!ok) break;
                 if (lane == 0) {
                     SegDesc &d = segs[slot];
-                    d.u = cur.a + j0;
+                    d.u = cur.a + r0;
                     d.s = cur.s;
                     d.h = cur.h;
                     d.j0 = j0;
@@ -496,11 +528,15 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     d.terminal = 0;
                     d.ksc = FP8 ? __ldg(p.k_scale + cur.h) : 1.f;
                     d.vsc = FP8 ? __ldg(p.v_scale + cur.h) : 1.f;
+                    d.jlo = cur.jlo;
                     const uint32_t bar = seg_full + 8 * slot;
-                    mbar_arrive_expect_tx(bar, qbytes);
-                    bulk_copy_g2s(sQ + slot * C::QSLOT,
-                                  p.q + ((long long)cur.s * p.num_q_heads + (long long)cur.h * g) * D,
-                                  qbytes, bar);
+                    mbar_arrive_expect_tx(bar, qtok * p.q_len);
+                    // query rows: q_len runs of g contiguous heads, row = i*g + head
+                    for (int i = 0; i < p.q_len; ++i)
+                        bulk_copy_g2s(sQ + slot * C::QSLOT + i * qtok,
+                                      p.q + (((long long)cur.s * p.q_len + i) * p.num_q_heads +
+                                             (long long)cur.h * g) * D,
+                                      qtok, bar);
                 }
                 ++sit;
             }
@@ -602,17 +638,32 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         const int terminal = (int)lds32(da + offsetof(SegDesc, terminal));
         const float ksc = __uint_as_float(lds32(da + offsetof(SegDesc, ksc)));
         const float vsc = __uint_as_float(lds32(da + offsetof(SegDesc, vsc)));
+        const int jlo = (int)lds32(da + offsetof(SegDesc, jlo));
         if (named_bar_sync_or(kBarConsumers, kConsumers, !seg_ok || terminal)) return;
-        const bool whole = (j0 == 0 && j1 == nunit);
+        const bool whole = (j0 == jlo && j1 == nunit);
+        const int R = p.rows;
 
-        // query fragments (B operand, Q^T[d][head]) from the slot
+        // visible token range [lo, hi) of the two query rows this lane holds
+        // per n-tile (rows 8*nt + 2*t4 + {0, 1}; row = query token * g + head)
+        int vis_lo[NT][2], vis_hi[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int row = nt * 8 + 2 * t4 + e;
+                const int hi = ctx - p.q_len + 1 + row / g;
+                vis_hi[nt][e] = row < R ? hi : 0;
+                vis_lo[nt][e] = (row < R && p.window > 0) ? max(0, hi - p.window) : 0;
+            }
+
+        // query fragments (B operand, Q^T[d][row]) from the slot
         uint32_t qf[C::KSTEPS][NT][2];
         {
             const uint32_t qb = sQ + qs * C::QSLOT;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                const int head = nt * 8 + gid;
-                const bool live = head < g;
+                const int head = nt * 8 + gid;      // query row held as B column
+                const bool live = head < R;
                 const uint32_t qr = qb + (live ? head : 0) * D * 2;
 #pragma unroll
                 for (int k = 0; k < C::KSTEPS; ++k) {
@@ -709,10 +760,16 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
+                    // stage token (only the first n_valid were loaded: the
+                    // stage may end with the segment, before the context
+                    // does) and its absolute position; the row's visible
+                    // range excludes padding rows and positions past ctx
                     const int tok = 16 * warp + gid + (e >> 1) * 8;
-                    const int head = nt * 8 + 2 * t4 + (e & 1);
+                    const int pos = jj * BS + tok;
                     const float v = sacc[nt][e] + sac2[nt][e];
-                    sacc[nt][e] = (tok < n_valid && head < g) ? v * sl2 : -INFINITY;
+                    sacc[nt][e] = (tok < n_valid && pos >= vis_lo[nt][e & 1] &&
+                                   pos < vis_hi[nt][e & 1])
+                                      ? v * sl2 : -INFINITY;
                 }
                 mx[nt][0] = fmaxf(sacc[nt][0], sacc[nt][2]);
                 mx[nt][1] = fmaxf(sacc[nt][1], sacc[nt][3]);
@@ -899,7 +956,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             if (!FP8) return C::DW * warp + 16 * mt + gid + (e >> 1) * 8;
             return 32 * warp + 4 * gid + 2 * mt + (e >> 1);
         };
-        const long long row0 = (long long)s * p.num_q_heads + (long long)h * g;
+        // output row of query row r: query token r / g, head h*g + r % g
+        auto orow = [&](int r) -> long long {
+            return ((long long)s * p.q_len + r / g) * p.num_q_heads + (long long)h * g + r % g;
+        };
         if (whole) {
 #pragma unroll
             for (int mt = 0; mt < C::MT; ++mt)
@@ -907,10 +967,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int head = nt * 8 + 2 * t4 + (e & 1);
-                        if (head < g) {
+                        const int r = nt * 8 + 2 * t4 + (e & 1);
+                        if (r < R) {
                             const float v = (o_hi[mt][nt][e] + o_lo[mt][nt][e]) * inv_l[nt][e & 1];
-                            p.out[(row0 + head) * D + dim_of(mt, e)] =
+                            p.out[orow(r) * D + dim_of(mt, e)] =
                                 __bfloat16_as_ushort(__float2bfloat16_rn(v));
                         }
                     }
@@ -919,24 +979,24 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int head = nt * 8 + 2 * t4 + e;
-                        if (head < g) p.lse_out[row0 + head] = lse2[nt][e] * kLn2;
+                        const int r = nt * 8 + 2 * t4 + e;
+                        if (r < R) p.lse_out[orow(r)] = lse2[nt][e] * kLn2;
                     }
             }
         } else {
             // partial: slot 2c for the CTA's first segment, 2c+1 for its last
             const bool first_seg = (useg == u0);
             const long long slot = 2 * cta + (first_seg ? 0 : 1);
-            float *op = p.o_part + slot * g * D;
+            float *op = p.o_part + slot * R * D;
 #pragma unroll
             for (int mt = 0; mt < C::MT; ++mt)
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int head = nt * 8 + 2 * t4 + (e & 1);
-                        if (head < g)
-                            op[head * D + dim_of(mt, e)] =
+                        const int r = nt * 8 + 2 * t4 + (e & 1);
+                        if (r < R)
+                            op[r * D + dim_of(mt, e)] =
                                 (o_hi[mt][nt][e] + o_lo[mt][nt][e]) * inv_l[nt][e & 1];
                     }
             if (warp == 0 && gid == 0) {
@@ -944,15 +1004,15 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int head = nt * 8 + 2 * t4 + e;
-                        if (head < g) p.lse_part[slot * g + head] = lse2[nt][e];
+                        const int r = nt * 8 + 2 * t4 + e;
+                        if (r < R) p.lse_part[slot * R + r] = lse2[nt][e];
                     }
             }
             __threadfence();
             named_bar_sync(kBarConsumers, kConsumers);
-            // unit tile range [ua, ub) and the CTAs that share it
-            const long long ua = useg - j0;   // flattened index of tile (s, h, 0)
-            const long long ub = ua + nunit;
+            // unit tile range [ua, ub) in work space and the CTAs that share it
+            const long long ua = useg - (j0 - jlo);
+            const long long ub = ua + (nunit - jlo);
             const long long c_first = cta_of(ua, U, G), c_last = cta_of(ub - 1, U, G);
             if (tid == 0) {
                 const int prev = atomicAdd(p.counters + (long long)s * Hkv + h, 1);
@@ -961,7 +1021,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             named_bar_sync(kBarConsumers, kConsumers);
             if (misc->is_last) {
                 __threadfence();
-                merge_unit<D>(p, ua, U, G, c_first, c_last, row0, g);
+                merge_unit<D>(p, ua, U, G, c_first, c_last, s, h);
                 if (tid == 0) p.counters[(long long)s * Hkv + h] = 0;
             }
         }

@@ -31,6 +31,9 @@ def lib():
     L.pgd_kv_append.argtypes = [P, P, P, i32, P, P, i32, i32, i32, i32, ctypes.c_int, P]
     L.pgd_paged_decode_attention.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32, i32,
                                              i32, f32, ctypes.c_int, P, P, P, P, P, sz, i32, P]
+    L.pgd_paged_decode_attention_ex.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32,
+                                                i32, i32, i32, i32, f32, ctypes.c_int, P, P, P, P,
+                                                P, sz, i32, P]
     L.pgd_merge_partials.argtypes = [P, P, i32, i32, i32, P, P, P]
     L.pgd_status_string.restype = ctypes.c_char_p
     L.pgd_version.restype = ctypes.c_char_p
@@ -80,7 +83,7 @@ def decode(lib, **kw):
 
 @pytest.mark.parametrize("kw,status", [
     (dict(Hq=6, Hkv=4), INVALID),          # heads not a multiple
-    (dict(Hq=24, Hkv=8), UNSUPPORTED),     # group 3
+    (dict(Hq=34, Hkv=2), UNSUPPORTED),     # group 17
     (dict(Hq=64, Hkv=2), UNSUPPORTED),     # group 32
     (dict(D=64), UNSUPPORTED),
     (dict(bs=8), UNSUPPORTED),
@@ -101,6 +104,32 @@ def decode(lib, **kw):
 ])
 def test_decode_host_validation(lib, kw, status):
     assert decode(lib, **kw) == status
+
+
+def decode_ex(lib, q_len, window, **kw):
+    args = dict(q=A, k=A, v=A, bt=A, mbps=8, cl=A, B=2, maxctx=0, Hq=8, Hkv=2, D=128, bs=16,
+                nb=16, scale=0.1, dt=0, ks=None, vs=None, out=A, lse=None, ws=None, wsb=0,
+                nctas=0)
+    args.update(kw)
+    a = args
+    return lib.pgd_paged_decode_attention_ex(a["q"], a["k"], a["v"], a["bt"], a["mbps"], a["cl"],
+                                             a["B"], a["maxctx"], q_len, window, a["Hq"],
+                                             a["Hkv"], a["D"], a["bs"], a["nb"], a["scale"],
+                                             a["dt"], a["ks"], a["vs"], a["out"], a["lse"],
+                                             a["ws"], a["wsb"], a["nctas"], None)
+
+
+@pytest.mark.parametrize("q_len,window,kw,status", [
+    (0, 0, {}, INVALID),                   # no query token
+    (1, -1, {}, INVALID),                  # negative window
+    (5, 0, {}, UNSUPPORTED),               # g * q_len = 20 rows > 16
+    (2, 0, dict(Hq=16, Hkv=1), UNSUPPORTED),
+    (4, 3, dict(out=MIS), INVALID),
+    (4, 3, dict(B=0, q=None), OK),
+    (8, 0, dict(Hq=4, Hkv=2, B=0), OK),    # 16 rows: accepted
+])
+def test_decode_ex_host_validation(lib, q_len, window, kw, status):
+    assert decode_ex(lib, q_len, window, **kw) == status
 
 
 @pytest.mark.parametrize("kw,status", [

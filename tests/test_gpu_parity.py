@@ -50,6 +50,9 @@ SHAPES = [  # (Hq, Hkv, D, bs, dtype)
     (16, 8, 256, 16, "bf16"), (32, 2, 128, 16, "bf16"), (64, 4, 256, 64, "bf16"),
     (64, 8, 128, 16, "e4m3"), (32, 2, 128, 32, "e4m3"), (8, 8, 128, 64, "e4m3"),
     (16, 1, 128, 16, "e4m3"),
+    # groups that are not powers of two (7: 28 query heads over 4 KV heads)
+    (28, 4, 128, 16, "bf16"), (12, 4, 128, 32, "e4m3"), (20, 2, 256, 64, "bf16"),
+    (5, 1, 128, 16, "bf16"),
 ]
 CTX = [1, 15, 16, 17, 63, 64, 65, 200, 1000, 2049, 0, 333]
 
