@@ -267,6 +267,57 @@ pgd_status pgd_paged_decode_attention_ex(
     void *out, float *lse_out,
     void *workspace, size_t workspace_bytes, int32_t num_ctas, void *stream);
 
+/* ------------------------------------------------------------------------ */
+/* KV parallelism: one sequence's KV split along its length over GPUs       */
+/* ------------------------------------------------------------------------ */
+/*
+ * Models with few KV heads run out of tensor parallelism at the KV head
+ * count; attention then shards each sequence's KV along its length over the
+ * GPUs (KVP, the co-design page's "Principle 4").  Each GPU decodes its
+ * slice into an unrounded split result (o, lse), the GPUs exchange those
+ * (an all-gather of num_seqs * num_q_heads * (head_dim + 1) fp32 per GPU),
+ * and pgd_merge_partials combines them exactly as the splits inside one GPU
+ * are combined ("attention kernels", "prefill and decode attention").
+ *
+ * pgd_kvp_plan -- host function (no CUDA call): the slice of every sequence
+ * that `rank` holds.  A sequence with nb = ceil(n / block_size) blocks is cut
+ * at block boundaries into world_size contiguous runs; rank r holds logical
+ * blocks [floor(nb * r / W), floor(nb * (r + 1) / W)), i.e. tokens from
+ * block_start[s] * block_size, slice_len[s] of them (0 when the run is
+ * empty).  The rank's block table lists those blocks in order, so its slice
+ * decodes as a sequence of slice_len[s] tokens.
+ *   context_lens  host int32 [num_seqs], each >= 0
+ *   block_start, slice_len  host int32 [num_seqs], written
+ *   world_size >= 1, 0 <= rank < world_size
+ */
+pgd_status pgd_kvp_plan(const int32_t *context_lens, int32_t num_seqs, int32_t block_size,
+                        int32_t world_size, int32_t rank, int32_t *block_start,
+                        int32_t *slice_len);
+
+/*
+ * pgd_paged_decode_partial -- pgd_paged_decode_attention for one KV slice,
+ * with the result left unrounded for a later merge: o_part gets the fp32
+ * softmax-weighted sum over the slice's tokens and lse_part its natural-log
+ * log-sum-exp (required).  A sequence with an empty slice gets o = 0 and
+ * lse = -inf, which carries no weight in the merge.
+ *
+ *   o_part    device fp32 [num_seqs][num_q_heads][head_dim], 16-byte aligned
+ *   lse_part  device fp32 [num_seqs][num_q_heads]
+ *   all other arguments, limits and errors as pgd_paged_decode_attention
+ *   (context_lens and block_table describe the slice).
+ * The outputs of W slices, stacked as [W][num_seqs * num_q_heads][head_dim]
+ * and [W][num_seqs * num_q_heads], are pgd_merge_partials' inputs.
+ */
+pgd_status pgd_paged_decode_partial(
+    const void *q, const void *k_cache, const void *v_cache,
+    const int32_t *block_table, int32_t max_blocks_per_seq,
+    const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t num_blocks, float scale, pgd_kv_dtype kv_dtype,
+    const float *k_scale, const float *v_scale,
+    float *o_part, float *lse_part,
+    void *workspace, size_t workspace_bytes, int32_t num_ctas, void *stream);
+
 /*
  * pgd_paged_decode_attention_noalloc -- the same decode step as
  * pgd_paged_decode_attention, for callers that must not have the library

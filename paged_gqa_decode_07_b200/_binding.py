@@ -12,6 +12,7 @@ import ctypes
 import os
 from typing import Optional
 
+import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -64,6 +65,11 @@ def load_library():
     lib.pgd_paged_decode_attention_ex.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32,
                                                   i32, i32, i32, i32, f32, st, P, P, P, P, P, sz,
                                                   i32, P]
+    lib.pgd_paged_decode_partial.restype = st
+    lib.pgd_paged_decode_partial.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32, i32,
+                                             i32, f32, st, P, P, P, P, P, sz, i32, P]
+    lib.pgd_kvp_plan.restype = st
+    lib.pgd_kvp_plan.argtypes = [P, i32, i32, i32, i32, P, P]
     lib.pgd_decode_step.restype = st
     lib.pgd_decode_step.argtypes = [P, P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, i32, i32,
                                     f32, st, P, P, P, P, P, sz, i32, P]
@@ -264,6 +270,65 @@ def paged_decode_attention_ex(q, k_cache, v_cache, block_table, context_lens, nu
         _ptr(out), _ptr(lse_out), _ptr(workspace), ws_bytes, int(num_ctas), _stream(stream)),
         "pgd_paged_decode_attention_ex")
     return out
+
+
+def paged_decode_partial(q, k_cache, v_cache, block_table, context_lens, num_q_heads: int,
+                         num_kv_heads: int, head_dim: int, block_size: int, scale: float,
+                         o_part: Optional[torch.Tensor] = None,
+                         lse_part: Optional[torch.Tensor] = None, *, max_context_len: int = 0,
+                         k_scale=None, v_scale=None, workspace=None, num_ctas: int = 0,
+                         stream=None):
+    """Decode of one KV slice left unrounded for a merge
+    (pgd_paged_decode_partial): returns (o_part fp32 [B][Hq][D],
+    lse_part fp32 [B][Hq], natural log)."""
+    lib = load_library()
+    _need(q, "q", (torch.bfloat16,), 3)
+    _need(k_cache, "k_cache", _KV_DTYPES, 4)
+    _need(v_cache, "v_cache", (k_cache.dtype,), 4)
+    _need(block_table, "block_table", (torch.int32,), 2)
+    _need(context_lens, "context_lens", (torch.int32,), 1)
+    B = q.shape[0]
+    if q.shape != (B, num_q_heads, head_dim) or tuple(k_cache.shape[1:]) != (
+            num_kv_heads, block_size, head_dim) or v_cache.shape != k_cache.shape or \
+            block_table.shape[0] != B or context_lens.shape[0] != B:
+        raise ValueError("paged_decode_partial: inconsistent shapes")
+    kvd = _kv_dtype(k_cache)
+    if kvd == PGD_KV_FP8_E4M3:
+        _need(k_scale, "k_scale", (torch.float32,), 1)
+        _need(v_scale, "v_scale", (torch.float32,), 1)
+    if o_part is None:
+        o_part = torch.empty((B, num_q_heads, head_dim), dtype=torch.float32, device=q.device)
+    if lse_part is None:
+        lse_part = torch.empty((B, num_q_heads), dtype=torch.float32, device=q.device)
+    _need(o_part, "o_part", (torch.float32,), 3)
+    _need(lse_part, "lse_part", (torch.float32,), 2)
+    if o_part.shape != (B, num_q_heads, head_dim) or lse_part.shape != (B, num_q_heads):
+        raise ValueError("paged_decode_partial: output shapes")
+    ws_bytes = 0
+    if workspace is not None:
+        _need(workspace, "workspace", None)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.pgd_paged_decode_partial(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), block_table.shape[1],
+        _ptr(context_lens), B, int(max_context_len), num_q_heads, num_kv_heads, head_dim,
+        block_size, k_cache.shape[0], float(scale), kvd, _ptr(k_scale), _ptr(v_scale),
+        _ptr(o_part), _ptr(lse_part), _ptr(workspace), ws_bytes, int(num_ctas), _stream(stream)),
+        "pgd_paged_decode_partial")
+    return o_part, lse_part
+
+
+def kvp_plan(context_lens, block_size: int, world_size: int, rank: int):
+    """Host-side KV-parallel slice of every sequence held by `rank`
+    (pgd_kvp_plan): returns (block_start, slice_len), int32 numpy [B]."""
+    lib = load_library()
+    cl = np.ascontiguousarray(np.asarray(context_lens, dtype=np.int32))
+    B = int(cl.shape[0])
+    start = np.zeros(B, np.int32)
+    length = np.zeros(B, np.int32)
+    _check(lib.pgd_kvp_plan(cl.ctypes.data_as(ctypes.c_void_p), B, int(block_size),
+                            int(world_size), int(rank), start.ctypes.data_as(ctypes.c_void_p),
+                            length.ctypes.data_as(ctypes.c_void_p)), "pgd_kvp_plan")
+    return start, length
 
 
 def decode_step(q, k_new, v_new, k_cache, v_cache, block_table, context_lens, num_q_heads: int,

@@ -4,6 +4,7 @@
 // pgd_get_device_error() and workspace growth.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstring>
@@ -273,7 +274,8 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
                        pgd_kv_dtype kv_dtype, const float *k_scale, const float *v_scale,
                        const void *k_new, const void *v_new, void *out, float *lse_out,
                        void *workspace, size_t workspace_bytes, int32_t num_ctas,
-                       void *stream, int32_t q_len = 1, int32_t window = 0) {
+                       void *stream, int32_t q_len = 1, int32_t window = 0,
+                       bool out_f32 = false) {
     // ---- host-side checks (nothing is enqueued on failure) ------------------
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
         max_blocks_per_seq <= 0 || max_context_len < 0 || num_ctas < 0 || q_len < 1 ||
@@ -389,6 +391,7 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     p.q_len = q_len;
     p.window = window;
     p.rows = rows;
+    p.out_f32 = out_f32 ? 1 : 0;
     a.grid = static_cast<int>(grid);
     a.stream = s;
     cudaError_t e = var.launch(a);
@@ -438,6 +441,41 @@ pgd_status pgd_paged_decode_attention_ex(
                        block_size, num_blocks, scale, kv_dtype, k_scale, v_scale, nullptr,
                        nullptr, out, lse_out, workspace, workspace_bytes, num_ctas, stream,
                        q_len, window);
+}
+
+pgd_status pgd_paged_decode_partial(
+    const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+    int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
+    int32_t max_context_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t num_blocks, float scale, pgd_kv_dtype kv_dtype,
+    const float *k_scale, const float *v_scale, float *o_part, float *lse_part, void *workspace,
+    size_t workspace_bytes, int32_t num_ctas, void *stream) {
+    if (num_seqs > 0 && !lse_part) return PGD_ERR_INVALID_ARG;
+    return decode_impl(q, k_cache, v_cache, block_table, max_blocks_per_seq, context_lens,
+                       num_seqs, max_context_len, num_q_heads, num_kv_heads, head_dim,
+                       block_size, num_blocks, scale, kv_dtype, k_scale, v_scale, nullptr,
+                       nullptr, o_part, lse_part, workspace, workspace_bytes, num_ctas, stream,
+                       1, 0, true);
+}
+
+pgd_status pgd_kvp_plan(const int32_t *context_lens, int32_t num_seqs, int32_t block_size,
+                        int32_t world_size, int32_t rank, int32_t *block_start,
+                        int32_t *slice_len) {
+    if (num_seqs < 0 || block_size <= 0 || world_size < 1 || rank < 0 || rank >= world_size)
+        return PGD_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PGD_OK;
+    if (!context_lens || !block_start || !slice_len) return PGD_ERR_INVALID_ARG;
+    for (int32_t s = 0; s < num_seqs; ++s)
+        if (context_lens[s] < 0) return PGD_ERR_INVALID_ARG;
+    for (int32_t s = 0; s < num_seqs; ++s) {
+        const long long n = context_lens[s];
+        const long long nb = (n + block_size - 1) / block_size;
+        const long long b0 = nb * rank / world_size, b1 = nb * (rank + 1) / world_size;
+        const long long t0 = b0 * block_size, t1 = std::min(n, b1 * block_size);
+        block_start[s] = static_cast<int32_t>(b0);
+        slice_len[s] = static_cast<int32_t>(t1 > t0 ? t1 - t0 : 0);
+    }
+    return PGD_OK;
 }
 
 pgd_status pgd_merge_partials(const float *o_part, const float *lse_part, int32_t num_parts,

@@ -50,7 +50,7 @@ namespace pgd {
 
 struct DecodeParams {
     const uint16_t *q;            // bf16 bits [B][Hq][D], 16-byte aligned
-    uint16_t *out;                // bf16 bits [B][Hq][D]
+    uint16_t *out;                // bf16 bits [B][Hq][D] (fp32 with out_f32)
     float *lse_out;               // [B][Hq] natural log, may be null
     const int32_t *block_table;   // [B][max_blocks_per_seq]
     const int32_t *context_lens;  // [B]
@@ -76,6 +76,9 @@ struct DecodeParams {
     // sequence with n tokens sits at position n - q_len + i and sees tokens
     // below n - q_len + 1 + i, and with window > 0 only the last window of them.
     int32_t q_len, window, rows;
+    // 1: out holds fp32 values (the unrounded split result a caller merges
+    // with other splits of the same rows); 0: bf16
+    int32_t out_f32;
 };
 
 constexpr int kConsumerWarps = 4;
@@ -338,10 +341,16 @@ __device__ __forceinline__ void merge_unit(const DecodeParams &p, long long ua, 
     for (int i = 0; i < MAXC; ++i) {
         const int col = sub + i * tph;
         if (col < V4) {
-            uint2 packed;
-            packed.x = pack_bf16x2(acc[i].x * inv, acc[i].y * inv);
-            packed.y = pack_bf16x2(acc[i].z * inv, acc[i].w * inv);
-            *reinterpret_cast<uint2 *>(p.out + orow * D + 4 * col) = packed;
+            if (p.out_f32) {
+                const float4 v =
+                    make_float4(acc[i].x * inv, acc[i].y * inv, acc[i].z * inv, acc[i].w * inv);
+                *reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + orow * D + 4 * col) = v;
+            } else {
+                uint2 packed;
+                packed.x = pack_bf16x2(acc[i].x * inv, acc[i].y * inv);
+                packed.y = pack_bf16x2(acc[i].z * inv, acc[i].w * inv);
+                *reinterpret_cast<uint2 *>(p.out + orow * D + 4 * col) = packed;
+            }
         }
     }
     if (p.lse_out && sub == 0)
@@ -420,8 +429,9 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         for (int i = 0; i < p.q_len; ++i) {
             const long long row0 =
                 ((long long)s * p.q_len + i) * p.num_q_heads + (long long)h * g;
-            uint16_t *o = p.out + row0 * D;
-            for (int e = 0; e < g * D; ++e) o[e] = 0;
+            const int words = p.out_f32 ? 2 * g * D : g * D;   // 16-bit words
+            uint16_t *o = p.out + row0 * D * (p.out_f32 ? 2 : 1);
+            for (int e = 0; e < words; ++e) o[e] = 0;
             if (p.lse_out)
                 for (int e = 0; e < g; ++e) p.lse_out[row0 + e] = -INFINITY;
         }
@@ -970,8 +980,9 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                         const int r = nt * 8 + 2 * t4 + (e & 1);
                         if (r < R) {
                             const float v = (o_hi[mt][nt][e] + o_lo[mt][nt][e]) * inv_l[nt][e & 1];
-                            p.out[orow(r) * D + dim_of(mt, e)] =
-                                __bfloat16_as_ushort(__float2bfloat16_rn(v));
+                            const long long at = orow(r) * D + dim_of(mt, e);
+                            if (p.out_f32) reinterpret_cast<float *>(p.out)[at] = v;
+                            else p.out[at] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
                         }
                     }
             if (p.lse_out && warp == 0 && gid == 0) {

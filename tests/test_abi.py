@@ -156,3 +156,14 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(b, "_lib", None)
     with pytest.raises(ImportError):
         b.load_library()
+
+
+def test_partial_decode_needs_lse(lib):
+    P, i32, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    lib.pgd_paged_decode_partial.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32, i32,
+                                             i32, f32, ctypes.c_int, P, P, P, P, P, sz, i32, P]
+    args = [A, A, A, A, 8, A, 2, 0, 8, 2, 128, 16, 16, 0.1, 0, None, None]
+    assert lib.pgd_paged_decode_partial(*args, A, None, None, 0, 0, None) == INVALID
+    assert lib.pgd_paged_decode_partial(*args, MIS, A, None, 0, 0, None) == INVALID
+    args[6] = 0   # empty batch
+    assert lib.pgd_paged_decode_partial(*args, None, None, None, 0, 0, None) == OK
