@@ -14,6 +14,15 @@ With N > 1 (torchrun) every rank runs its own independent batch (weak
 scaling, no collective on the data path); time is the max over ranks.
 
 --impl reference times the fp64 CPU oracle on host cores (rank 0 only).
+
+Other rows of the path, same JSON line, each on its own workload shape:
+    --q-len L --window W   decode of the L newest tokens per sequence (causal
+                           among them) and/or a sliding window of W tokens
+                           (pgd_paged_decode_attention_ex); the bytes count
+                           the visible K/V rows only
+    --kvp                  one batch with every sequence's KV split along its
+                           length over the N ranks: slice decode to fp32,
+                           all-gather, log-sum-exp merge (strong scaling)
 """
 from __future__ import annotations
 
@@ -179,6 +188,177 @@ def reduce_over_ranks(step_bytes: int, ms_step: float, e2e_ms: float, dec_ms: fl
 # --------------------------------------------------------------------------- #
 # our arm                                                                     #
 # --------------------------------------------------------------------------- #
+def _to_torch(a, dev=None, pin=False):
+    """numpy -> torch (bf16 bits stay bf16); pinned host memory or `dev`."""
+    import torch
+    a = np.ascontiguousarray(a)
+    t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+    if a.dtype == np.uint16:
+        t = t.view(torch.bfloat16)
+    return t.pin_memory() if pin else t.to(dev)
+
+
+class Mode:
+    """One kind of timed step.  step(inp, ev) runs one step on the tensors of
+    `inp` (device resident); with `ev` = (start, end) events it records them
+    around the dominant kernel's launch."""
+    single = True            # one launch per step: its duration = region / K
+    kernel = "paged_decode_kernel"
+    scaling = "weak"
+
+    def __init__(self):
+        self.inputs, self.host, self.out = {}, {}, None
+        self.cfg = {}
+
+
+def mode_step(args, w, pgd, dev, stream):
+    """The decode step: kv_append of each sequence's newest token fused into
+    the decode launch (pgd_decode_step), or --unfused: the two calls."""
+    m = Mode()
+    T = lambda a: _to_torch(a, dev)  # noqa: E731
+    k, v = T(w.k_cache), T(w.v_cache)
+    ks = T(w.k_scale) if w.k_scale is not None else None
+    vs = T(w.v_scale) if w.v_scale is not None else None
+    has_app = w.slot_mapping is not None
+    arrays = {"q": w.q, "bt": w.block_table, "cl": w.context_lens}
+    if has_app:
+        arrays.update(kn=w.k_new, vn=w.v_new, sl=w.slot_mapping)
+    m.inputs = {n: T(a) for n, a in arrays.items()}
+    m.host = {n: _to_torch(a, pin=True) for n, a in arrays.items()}
+    m.out = torch_empty_like(m.inputs["q"])
+    fused = has_app and not args.unfused and len(w.slot_mapping) == w.num_seqs
+    mcl = w.max_context_len
+    ab = w.algorithmic_bytes()
+
+    def decode(inp):
+        if fused:
+            pgd.decode_step(inp["q"], inp["kn"], inp["vn"], k, v, inp["bt"], inp["cl"],
+                            w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, w.scale,
+                            m.out, max_context_len=mcl, k_scale=ks, v_scale=vs, stream=stream)
+        else:
+            pgd.paged_decode_attention(inp["q"], k, v, inp["bt"], inp["cl"], w.num_q_heads,
+                                       w.num_kv_heads, w.head_dim, w.block_size, w.scale, m.out,
+                                       max_context_len=mcl, k_scale=ks, v_scale=vs,
+                                       stream=stream)
+
+    def step(inp, ev=None):
+        if has_app and not fused:
+            pgd.kv_append(inp["kn"], inp["vn"], inp["sl"], k, v, stream=stream)
+        if ev:
+            ev[0].record(stream)
+        decode(inp)
+        if ev:
+            ev[1].record(stream)
+
+    m.step = step
+    m.single = fused or not has_app
+    m.launches = 2 if has_app and not fused else 1
+    m.kernel = "paged_decode_kernel" + (" (fused append)" if fused else "")
+    m.dec_bytes = ab["step_total"] if fused else ab["decode_total"]
+    m.step_bytes = ab["step_total"]
+    m.fused = fused
+    return m
+
+
+def mode_ex(args, w, pgd, dev, stream):
+    """q_len query tokens per sequence and/or a sliding window
+    (pgd_paged_decode_attention_ex).  The append payload, if the workload
+    has one, is written once before timing, so every token is cached."""
+    from workloads import multi_query
+    m = Mode()
+    T = lambda a: _to_torch(a, dev)  # noqa: E731
+    k, v = T(w.k_cache), T(w.v_cache)
+    ks = T(w.k_scale) if w.k_scale is not None else None
+    vs = T(w.v_scale) if w.v_scale is not None else None
+    if w.slot_mapping is not None:
+        pgd.kv_append(T(w.k_new), T(w.v_new), T(w.slot_mapping), k, v, stream=stream)
+    L, W = args.q_len, args.window
+    arrays = {"q": multi_query(w, L, seed=0), "bt": w.block_table, "cl": w.context_lens}
+    m.inputs = {n: T(a) for n, a in arrays.items()}
+    m.host = {n: _to_torch(a, pin=True) for n, a in arrays.items()}
+    m.out = torch_empty_like(m.inputs["q"])
+    mcl = w.max_context_len
+
+    def step(inp, ev=None):
+        if ev:
+            ev[0].record(stream)
+        pgd.paged_decode_attention_ex(inp["q"], k, v, inp["bt"], inp["cl"], w.num_q_heads,
+                                      w.num_kv_heads, w.head_dim, w.block_size, w.scale, m.out,
+                                      window=W, max_context_len=mcl, k_scale=ks, v_scale=vs,
+                                      stream=stream)
+        if ev:
+            ev[1].record(stream)
+
+    ab = w.algorithmic_bytes(L, W)
+    m.step, m.launches, m.fused = step, 1, False
+    m.kernel = f"paged_decode_kernel (q_len {L}, window {W})"
+    m.dec_bytes = m.step_bytes = ab["decode_total"]
+    m.cfg = {"q_len": L, "window": W, "visible_tokens":
+             int(sum(b - a for a, b in zip(*w.visible_ranges(L, W))))}
+    return m
+
+
+def mode_kvp(args, w, pgd, dev, stream, rank, world):
+    """KV parallelism: every sequence's KV is split along its length over the
+    ranks (pgd_kvp_plan); a step is this rank's slice decode
+    (pgd_paged_decode_partial), the all-gather of the split results and the
+    merge (pgd_merge_partials).  Total work is fixed as ranks are added."""
+    import torch
+
+    from paged_gqa_decode_07_b200 import kvp
+    m = Mode()
+    T = lambda a: _to_torch(a, dev)  # noqa: E731
+    if w.slot_mapping is not None:
+        raise SystemExit("--kvp needs a workload without an append payload")
+    k, v = T(w.k_cache), T(w.v_cache)
+    ks = T(w.k_scale) if w.k_scale is not None else None
+    vs = T(w.v_scale) if w.v_scale is not None else None
+    start, length = kvp.plan(w.context_lens, w.block_size, world, rank)
+    table = kvp.local_block_table(w.block_table, start, length, w.block_size)
+    arrays = {"q": w.q, "bt": table, "cl": length}
+    m.inputs = {n: T(a) for n, a in arrays.items()}
+    m.host = {n: _to_torch(a, pin=True) for n, a in arrays.items()}
+    dec = kvp.KVPDecoder(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
+                         device=dev)
+    m.out = dec.out
+    mcl = int(length.max(initial=0))
+    rows = w.num_seqs * w.num_q_heads
+
+    def step(inp, ev=None):
+        if ev:
+            ev[0].record(stream)
+        pgd.paged_decode_partial(inp["q"], k, v, inp["bt"], inp["cl"], w.num_q_heads,
+                                 w.num_kv_heads, w.head_dim, w.block_size, w.scale,
+                                 dec.o_local, dec.lse_local, max_context_len=mcl, k_scale=ks,
+                                 v_scale=vs, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        kvp.gather_partials(dec.o_local, dec.lse_local, dec.o_all, dec.lse_all)
+        pgd.merge_partials(dec.o_all, dec.lse_all, dec.out.view(rows, w.head_dim), dec.lse,
+                           stream=stream)
+
+    bs, Hkv, D, e = w.block_size, w.num_kv_heads, w.head_dim, w.elem_bytes
+    blocks = int(((length.astype(np.int64) + bs - 1) // bs).sum())
+    slice_kv = int(length.astype(np.int64).sum()) * Hkv * D * 2 * e
+    meta = blocks * 4 + w.num_seqs * 4 + (2 * Hkv * 4 if w.kv_dtype == "e4m3" else 0)
+    # the slice kernel reads q, its slice and metadata, and writes fp32 o + lse
+    m.dec_bytes = slice_kv + meta + rows * D * 2 + rows * (D + 1) * 4
+    full = w.algorithmic_bytes()
+    # the job's bytes: every K/V row once, q in and out back once, metadata
+    m.step_bytes = slice_kv + meta + (full["qo"] if rank == 0 else 0)
+    m.step, m.single, m.launches, m.fused = step, False, 2, False
+    m.kernel = "paged_decode_kernel (fp32 split result of the rank's KV slice)"
+    m.scaling = "strong"
+    m.cfg = {"kvp_ranks": world, "exchange_bytes_per_rank": dec.exchange_bytes(),
+             "slice_tokens_this_rank": int(length.sum())}
+    return m
+
+
+def torch_empty_like(t):
+    import torch
+    return torch.empty_like(t)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -188,44 +368,19 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    # every rank runs its own batch: same shape (context lengths of seed 0),
-    # its own block permutation and values
-    w = make_workload(args.workload, seed=rank, shape_seed=0)
-    ab = w.algorithmic_bytes()
-
-    def to_dev(a, pin=False):
-        import numpy as _np
-        t = torch.from_numpy(_np.ascontiguousarray(a).view(_np.int16) if a.dtype == _np.uint16
-                             else _np.ascontiguousarray(a))
-        if a.dtype == np.uint16:
-            t = t.view(torch.bfloat16)
-        return t.pin_memory() if pin else t.to(dev)
-
-    q, k, v = to_dev(w.q), to_dev(w.k_cache), to_dev(w.v_cache)
-    bt, cl = to_dev(w.block_table), to_dev(w.context_lens)
-    ks = to_dev(w.k_scale) if w.k_scale is not None else None
-    vs = to_dev(w.v_scale) if w.v_scale is not None else None
-    has_app = w.slot_mapping is not None
-    if has_app:
-        kn, vn, sl = to_dev(w.k_new), to_dev(w.v_new), to_dev(w.slot_mapping)
-    out = torch.empty_like(q)
-    mcl = w.max_context_len
     stream = torch.cuda.current_stream()
-    # a decode step whose appended tokens are each sequence's newest token runs
-    # as one fused launch (pgd_decode_step); --unfused times append + decode
-    fused = has_app and not args.unfused and len(w.slot_mapping) == w.num_seqs
-
-    def step(q_, kn_, vn_, sl_, bt_, cl_, out_):
-        if fused:
-            pgd.decode_step(q_, kn_, vn_, k, v, bt_, cl_, w.num_q_heads, w.num_kv_heads,
-                            w.head_dim, w.block_size, w.scale, out_, max_context_len=mcl,
-                            k_scale=ks, v_scale=vs, stream=stream)
-            return
-        if has_app:
-            pgd.kv_append(kn_, vn_, sl_, k, v, stream=stream)
-        pgd.paged_decode_attention(q_, k, v, bt_, cl_, w.num_q_heads, w.num_kv_heads,
-                                   w.head_dim, w.block_size, w.scale, out_,
-                                   max_context_len=mcl, k_scale=ks, v_scale=vs, stream=stream)
+    if args.kvp:
+        # one batch split over the ranks: the same data on every rank
+        w = make_workload(args.workload, seed=0, shape_seed=0)
+        m = mode_kvp(args, w, pgd, dev, stream, rank, world)
+    else:
+        # every rank runs its own batch: same shape (context lengths of seed
+        # 0), its own block permutation and values
+        w = make_workload(args.workload, seed=rank, shape_seed=0)
+        if args.q_len > 1 or args.window > 0:
+            m = mode_ex(args, w, pgd, dev, stream)
+        else:
+            m = mode_step(args, w, pgd, dev, stream)
 
     def barrier():
         if world > 1:
@@ -233,31 +388,18 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- warm-up -------------------------------------------------------------
     for _ in range(args.warmup):
-        step(q, kn if has_app else None, vn if has_app else None, sl if has_app else None,
-             bt, cl, out)
+        m.step(m.inputs)
     torch.cuda.synchronize()
     assert pgd.get_device_error() == 0
 
-    def decode_only():
-        if fused:
-            pgd.decode_step(q, kn, vn, k, v, bt, cl, w.num_q_heads, w.num_kv_heads, w.head_dim,
-                            w.block_size, w.scale, out, max_context_len=mcl, k_scale=ks,
-                            v_scale=vs, stream=stream)
-        else:
-            pgd.paged_decode_attention(q, k, v, bt, cl, w.num_q_heads, w.num_kv_heads,
-                                       w.head_dim, w.block_size, w.scale, out,
-                                       max_context_len=mcl, k_scale=ks, v_scale=vs,
-                                       stream=stream)
-
     # ---- timed region: K back-to-back steps, device time ---------------------
-    # No event sits between launches (an event between two launches stops the
-    # next launch from overlapping its set-up with the previous one's tail).
-    # With one launch per step the decode kernel's average launch duration is
-    # this region's time / K; the unfused mode brackets each decode launch.
+    # No event sits between launches of a one-launch step (an event between
+    # two launches stops the next launch from overlapping its set-up with the
+    # previous one's tail): the kernel's average launch duration is this
+    # region's time / K.  Steps of several launches bracket the dominant one.
     K = args.steps
-    single = fused or not has_app          # one launch per step
-    ev_dec = [] if single else [(torch.cuda.Event(enable_timing=True),
-                                 torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ev_dec = [] if m.single else [(torch.cuda.Event(enable_timing=True),
+                                   torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     clocks = ClockSampler(local_rank) if not args.no_clocks else None
     if clocks:
         clocks.start()
@@ -268,55 +410,40 @@ def run_ours(args, rank, world, local_rank):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(K):
-        if single:
-            decode_only()
-            continue
-        pgd.kv_append(kn, vn, sl, k, v, stream=stream)
-        ev_dec[i][0].record(stream)
-        decode_only()
-        ev_dec[i][1].record(stream)
+        m.step(m.inputs, None if m.single else ev_dec[i])
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     t_end = time.time()
     clk = clocks.stop(t_begin, t_end) if clocks else None
     ms_total = e0.elapsed_time(e1)
-    if single:
+    if m.single:
         dec_avg_ms = ms_total / K
     else:
         dec_avg_ms = sum(a.elapsed_time(b) for a, b in ev_dec) / K
     flags = pgd.get_device_error()
-    # for reference: the same launch bracketed by its own events, one at a time
+    # for reference: the dominant launch bracketed by its own events, one at a time
     iso = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(min(K, 50))]
-    for a_, b_ in iso:
-        a_.record(stream)
-        decode_only()
-        b_.record(stream)
+    for ev in iso:
+        m.step(m.inputs, ev)
     torch.cuda.synchronize()
     iso_ms = sum(a_.elapsed_time(b_) for a_, b_ in iso) / len(iso)
 
     # ---- end to end through the public API with host buffers ----------------
-    hq = to_dev(w.q, pin=True)
-    hbt, hcl = to_dev(w.block_table, pin=True), to_dev(w.context_lens, pin=True)
-    dq, dbt, dcl = torch.empty_like(q), torch.empty_like(bt), torch.empty_like(cl)
-    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    h2d = [(hq, dq), (hbt, dbt), (hcl, dcl)]
-    if has_app:
-        hkn, hvn, hsl = to_dev(w.k_new, pin=True), to_dev(w.v_new, pin=True), \
-            to_dev(w.slot_mapping, pin=True)
-        dkn, dvn, dsl = torch.empty_like(kn), torch.empty_like(vn), torch.empty_like(sl)
-        h2d += [(hkn, dkn), (hvn, dvn), (hsl, dsl)]
-    h2d_bytes = sum(h.numel() * h.element_size() for h, _ in h2d)
+    # every step copies its inputs from pinned host memory and reads the
+    # output back
+    dinp = {n: torch.empty_like(t) for n, t in m.inputs.items()}
+    hout = torch.empty(m.out.shape, dtype=m.out.dtype, pin_memory=True)
+    h2d_bytes = sum(h.numel() * h.element_size() for h in m.host.values())
     d2h_bytes = hout.numel() * hout.element_size()
     Ke = max(1, min(K, args.e2e_steps))
 
     def e2e_step():
-        for h, d in h2d:
-            d.copy_(h, non_blocking=True)
-        step(dq, dkn if has_app else None, dvn if has_app else None, dsl if has_app else None,
-             dbt, dcl, out)
-        hout.copy_(out, non_blocking=True)
+        for n, h in m.host.items():
+            dinp[n].copy_(h, non_blocking=True)
+        m.step(dinp)
+        hout.copy_(m.out, non_blocking=True)
 
     for _ in range(3):
         e2e_step()
@@ -335,12 +462,12 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- aggregate over ranks ----------------------------------------------------
     ms_step = ms_total / K
-    agg = reduce_over_ranks(ab["step_total"], ms_step, e2e_ms, dec_avg_ms, world, dev)
-    ms_step, e2e_ms, dec_avg_ms = agg["ms_step"], agg["e2e_ms"], agg["dec_ms"]
+    agg = reduce_over_ranks(m.step_bytes, ms_step, e2e_ms, dec_avg_ms, world, dev)
+    ms_step, e2e_ms = agg["ms_step"], agg["e2e_ms"]
     value, e2e_value = agg["value"], agg["e2e_value"]
     peak, peak_kind = measured_peak()
-    dec_bytes = ab["step_total"] if fused else ab["decode_total"]
-    achieved = dec_bytes / (dec_avg_ms * 1e-3) / 1e9
+    # the dominant kernel of this rank (rank 0 prints its own launch figures)
+    achieved = m.dec_bytes / (dec_avg_ms * 1e-3) / 1e9
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -348,38 +475,42 @@ def run_ours(args, rank, world, local_rank):
 
     if rank == 0:
         cfg = workload_desc(w)
-        cfg.update({"parallelism": f"replicas x{world} (independent batch per GPU)",
-                    "l2": f"inputs larger than L2 ({ab['kv'] / 1e6:.0f} MB of KV read per step "
+        cfg.update(m.cfg)
+        kv_mb = w.algorithmic_bytes(max(1, args.q_len), args.window)["kv"] / 1e6
+        cfg.update({"parallelism": (f"KV parallel over {world} rank(s) (one batch, each "
+                                    f"sequence split along its length)") if args.kvp else
+                    f"replicas x{world} (independent batch per GPU)",
+                    "l2": f"inputs larger than L2 ({kv_mb:.0f} MB of KV read per step "
                           f"vs {L2_BYTES / 2**20:.0f} MiB L2); no flush",
-                    "global_batch": w.num_seqs * world})
+                    "global_batch": w.num_seqs * (1 if args.kvp else world)})
+        default_mode = not args.kvp and args.q_len == 1 and args.window == 0
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
             "us_per_step": round(ms_step * 1e3, 2),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True, "scaling": m.scaling, "vs_baseline": None,
             "dtype": w.kv_dtype, "data": "synthetic (seeded N(0,1) Q/K/V, shuffled block table)",
             "config": cfg,
             "pct_of_measured_hbm": round(100 * value / world / peak, 1),
             "pct_of_nominal_8tbs": round(100 * value / world / 8000.0, 1),
-            "roofline": {"bound": "hbm",
-                         "kernel": "paged_decode_kernel" + (" (fused append)" if fused else ""),
+            "roofline": {"bound": "hbm", "kernel": m.kernel,
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_kind == "measured" else "fallback 6.65 TB/s",
-                         "algorithmic_bytes_per_launch": dec_bytes,
+                         "algorithmic_bytes_per_launch": m.dec_bytes,
                          "avg_launch_us": round(dec_avg_ms * 1e3, 2),
                          "launch_timing": "timed region / K (one launch per step, "
-                                          "back to back)" if single else
-                                          "events around each decode launch",
+                                          "back to back)" if m.single else
+                                          "events around each dominant launch",
                          "isolated_launch_us": round(iso_ms * 1e3, 2),
-                         "traffic": recorded_traffic(args.workload)},
+                         "traffic": recorded_traffic(args.workload) if default_mode else None},
             "e2e": {"value": round(e2e_value, 1), "unit": "GB/s",
                     "us_per_step": round(e2e_ms * 1e3, 2),
                     "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
                     "steps": Ke},
-            "gpu_launches": K * (2 if has_app and not fused else 1),
-            "fused_step": fused,
+            "gpu_launches": K * m.launches,
+            "fused_step": m.fused,
             "clocks": clk,
             "device_flags": flags,
             "cpu_baseline": cpu,
@@ -497,9 +628,19 @@ def main():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--unfused", action="store_true",
                     help="time kv_append and the decode as two launches")
+    ap.add_argument("--q-len", type=int, default=1,
+                    help="query tokens per sequence (causal among them)")
+    ap.add_argument("--window", type=int, default=0,
+                    help="sliding window in tokens (0 = whole context)")
+    ap.add_argument("--kvp", action="store_true",
+                    help="split every sequence's KV over the ranks (strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.q_len < 1 or args.window < 0:
+        ap.error("--q-len must be >= 1 and --window >= 0")
+    if args.kvp and (args.q_len > 1 or args.window > 0 or args.unfused):
+        ap.error("--kvp runs the one-token decode without append")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -93,16 +93,27 @@ class Workload:
     def num_tokens(self) -> int:
         return int(self.context_lens.astype(np.int64).sum())
 
-    def algorithmic_bytes(self) -> dict:
+    def visible_ranges(self, q_len: int = 1, window: int = 0):
+        """Per sequence, the positions [lo, n) that some query row sees when
+        the q_len newest tokens are queried (token j sees positions below
+        n - q_len + 1 + j) with an optional window of `window` positions."""
+        n = self.context_lens.astype(np.int64)
+        if window <= 0:
+            return np.zeros_like(n), n
+        return np.maximum(0, n - q_len + 1 - window), n
+
+    def algorithmic_bytes(self, q_len: int = 1, window: int = 0) -> dict:
         """Bytes one decode step must move at minimum (see the design notes):
-        every cached K and V row once per (sequence, KV head), Q in, out back,
-        the block-table entries read, the context lengths, the FP8 scales and,
-        when present, the append payload read and written."""
+        every visible K and V row once per (sequence, KV head), Q in, out back,
+        the block-table entries of the visible blocks, the context lengths,
+        the FP8 scales and, when present, the append payload read and
+        written."""
         B, Hq, Hkv, D = self.num_seqs, self.num_q_heads, self.num_kv_heads, self.head_dim
-        kv = self.num_tokens * Hkv * D * 2 * self.elem_bytes
-        blocks = int(((self.context_lens.astype(np.int64) + self.block_size - 1)
-                      // self.block_size).sum())
-        qo = 2 * B * Hq * D * 2
+        lo, n = self.visible_ranges(q_len, window)
+        kv = int((n - lo).sum()) * Hkv * D * 2 * self.elem_bytes
+        bs = self.block_size
+        blocks = int(np.where(n > lo, (n - 1) // bs - lo // bs + 1, 0).sum())
+        qo = 2 * B * q_len * Hq * D * 2
         meta = blocks * 4 + B * 4 + (2 * Hkv * 4 if self.kv_dtype == "e4m3" else 0)
         app = 0
         if self.slot_mapping is not None and len(self.slot_mapping):
@@ -113,6 +124,14 @@ class Workload:
 
     def flops(self) -> int:
         return 4 * self.num_q_heads * self.head_dim * self.num_tokens
+
+
+def multi_query(w: Workload, q_len: int, seed: int = 0) -> np.ndarray:
+    """Query rows for q_len tokens per sequence, bf16 bits [B][q_len][Hq][D],
+    N(0, 1) from np.random.default_rng(seed + 7_000_001)."""
+    rng = np.random.default_rng(seed + 7_000_001)
+    return to_bf16_bits(rng.standard_normal((w.num_seqs, q_len, w.num_q_heads, w.head_dim),
+                                            dtype=np.float32))
 
 
 def _assign_blocks(rng, ctx: np.ndarray, bs: int, pool: int):
