@@ -210,17 +210,32 @@ __device__ __forceinline__ int first_block(int ctx, const DecodeParams &p) {
     return max(0, ctx - p.q_len + 1 - p.window) / BS;
 }
 
-// Walk over the units of a CTA's work range (producer and appender).  Unit
-// (s, h) reads blocks jlo .. n-1 and occupies work indices [a, a + w): its
-// n - jlo tiles first, then the fixed-cost slots, which hold no tiles.
+// Walk over the units of a CTA's work range (producer and appender; every
+// lane of the warp walks in step).  Unit (s, h) reads blocks jlo .. n-1 and
+// occupies work indices [a, a + w): its n - jlo tiles first, then the
+// fixed-cost slots, which hold no tiles.  The context lengths of 32
+// consecutive sequences sit one per lane (wbase, wval) and are read by
+// shuffle, so the walk issues one coalesced load per 32 sequences instead of
+// a dependent load per sequence.
 struct Cursor {
     int s, h, n, ctx, jlo;
     long long a, w;
+    int wbase, wval;
 };
 
 template <int BS>
+__device__ __forceinline__ int window_ctx(Cursor &c, const DecodeParams &p, int s) {
+    const int lane = threadIdx.x & 31;
+    if (s < c.wbase || s >= c.wbase + 32) {
+        c.wbase = s;
+        c.wval = s + lane < p.num_seqs ? ctx_of<BS>(p, s + lane) : 0;
+    }
+    return __shfl_sync(0xffffffffu, c.wval, s - c.wbase);
+}
+
+template <int BS>
 __device__ __forceinline__ void set_seq(Cursor &c, const DecodeParams &p) {
-    c.ctx = ctx_of<BS>(p, c.s);
+    c.ctx = window_ctx<BS>(c, p, c.s);
     c.n = nblk_of<BS>(c.ctx);
     c.jlo = first_block<BS>(c.ctx, p);
     c.w = unit_weight(c.n - c.jlo, p.unit_cost);
@@ -243,6 +258,8 @@ __device__ __forceinline__ Cursor first_unit(const DecodeParams &p, int s0, long
                                             long long u0) {
     Cursor c;
     c.s = s0;
+    c.wbase = -64;                   // empty window: the first read loads it
+    c.wval = 0;
     set_seq<BS>(c, p);
     c.h = (int)((u0 - pfx0) / c.w);
     c.a = pfx0 + (long long)c.h * c.w;
@@ -514,11 +531,56 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         const uint32_t qtok = (uint32_t)(g * D * 2);          // one query token's rows
         uint32_t it = 0, sit = 0, ait = 0;
         bool ok = true;
-        for (; cur.a < u1 && ok; next_unit<BS>(cur, p)) {
-            const int r0 = (int)max(0LL, u0 - cur.a);
-            const int r1 = (int)min((long long)(cur.n - cur.jlo), u1 - cur.a);
-            if (r0 >= r1) continue;   // the range holds only this unit's fixed-cost slots
-            const int j0 = cur.jlo + r0, j1 = cur.jlo + r1;   // absolute blocks
+        // FP8 scales of the first 32 KV heads, one per lane
+        float ks_l = 1.f, vs_l = 1.f;
+        if (FP8 && lane < Hkv) {
+            ks_l = __ldg(p.k_scale + lane);
+            vs_l = __ldg(p.v_scale + lane);
+        }
+        // the segment's blocks [j0, j1) of unit c (empty: only fixed-cost slots)
+        auto seg_of = [&](const Cursor &c, int &j0, int &j1) {
+            j0 = c.jlo + (int)max(0LL, u0 - c.a);
+            j1 = c.jlo + (int)min((long long)(c.n - c.jlo), u1 - c.a);
+        };
+        // block ids of a segment's first 32 blocks, one per lane; the next
+        // unit's are loaded while this unit's tiles are issued, so the walk
+        // never waits on a dependent block-table load
+        auto first_ids = [&](const Cursor &c, int j0, int j1) -> int {
+            const int32_t *bt = p.block_table + (long long)c.s * p.max_blocks_per_seq;
+            return j0 + lane < j1 ? __ldg(bt + j0 + lane) : 0;
+        };
+        int pf = 0;
+        if (cur.a < u1) {
+            int a0, a1;
+            seg_of(cur, a0, a1);
+            pf = first_ids(cur, a0, a1);
+        }
+        for (; cur.a < u1 && ok;) {
+            int j0, j1;                                  // absolute blocks
+            seg_of(cur, j0, j1);
+            Cursor nxt = cur;
+            next_unit<BS>(nxt, p);
+            int pf_next = 0;
+            if (nxt.a < u1) {
+                int b0, b1;
+                seg_of(nxt, b0, b1);
+                pf_next = first_ids(nxt, b0, b1);
+            }
+            if (j0 >= j1) {          // the range holds only this unit's fixed-cost slots
+                cur = nxt;
+                pf = pf_next;
+                continue;
+            }
+            const int r0 = j0 - cur.jlo;
+            float ksc = 1.f, vsc = 1.f;
+            if (FP8) {
+                ksc = __shfl_sync(0xffffffffu, ks_l, cur.h & 31);
+                vsc = __shfl_sync(0xffffffffu, vs_l, cur.h & 31);
+                if (cur.h >= 32) {
+                    ksc = __ldg(p.k_scale + cur.h);
+                    vsc = __ldg(p.v_scale + cur.h);
+                }
+            }
             // -- descriptor and query rows of the segment
             {
                 const uint32_t slot = sit % C::NSEG;
@@ -536,8 +598,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     d.n = cur.n;
                     d.ctx = cur.ctx;
                     d.terminal = 0;
-                    d.ksc = FP8 ? __ldg(p.k_scale + cur.h) : 1.f;
-                    d.vsc = FP8 ? __ldg(p.v_scale + cur.h) : 1.f;
+                    d.ksc = ksc;
+                    d.vsc = vsc;
                     d.jlo = cur.jlo;
                     const uint32_t bar = seg_full + 8 * slot;
                     mbar_arrive_expect_tx(bar, qtok * p.q_len);
@@ -556,7 +618,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             // -- K/V tiles, block ids fetched 32 at a time (one chunk ahead)
             const int32_t *bt = p.block_table + (long long)cur.s * p.max_blocks_per_seq;
             int jc = j0;
-            int pb_next = jc + lane < j1 ? __ldg(bt + jc + lane) : 0;
+            int pb_next = pf;
             while (jc < j1 && ok) {
                 const int pb_cur = pb_next;
                 const int jn = jc + 32;
@@ -596,6 +658,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 }
                 jc = jn;
             }
+            cur = nxt;
+            pf = pf_next;
         }
         if (!ok && lane == 0) raise_flag(p.flags, kFlagTimeout);
         if (lane == 0) {
