@@ -107,20 +107,23 @@ struct DecodeCfg {
     static constexpr int BPS = kStageTokens / BS;        // blocks per stage
     static constexpr int STAGE_KV = BPS * TILE;          // K (or V) bytes per stage
     static constexpr int STAGE = 2 * STAGE_KV;
-    static constexpr int NP = 8 * NT;                    // padded heads per unit
-    static constexpr int DW = D / kConsumerWarps;        // PV dims per warp
-    static constexpr int MT = DW / 16;                   // PV m-tiles per warp
+    static constexpr int NP = 8 * NT;                    // padded query rows per unit
+    static constexpr int DT = D / 16;                    // PV m-tiles (each warp: all of D)
     static constexpr int KSTEPS = D / 16;                // QK k-steps
     static constexpr int QSLOT = NP * D * 2;             // query rows of one unit
-    static constexpr int NSEG = QSLOT >= 4096 ? 2 : 4;   // descriptor ring depth
+    // descriptor ring depth (one slot for 16 query rows at head_dim 128, so
+    // that two CTAs still fit on an SM)
+    static constexpr int NSEG = D == 128 ? (QSLOT >= 4096 ? 1 : 3) : 2;
+    static constexpr int OROW = D + 4;                   // sO row stride in floats
     // shared memory carve-up (offsets from a 1024-aligned base)
-    static constexpr int P_BYTES = kStageTokens * NP * 2;   // one weight plane
-    static constexpr int OFF_P = NSTAGES * STAGE;
-    static constexpr int OFF_Q = OFF_P + 2 * P_BYTES;        // hi and lo planes
+    static constexpr int OFF_O = NSTAGES * STAGE;        // two 8-row O buffers
+    static constexpr int OBUF = 8 * OROW * 4;
+    static constexpr int OFF_Q = OFF_O + 2 * OBUF;
     static constexpr int OFF_SEG = OFF_Q + NSEG * QSLOT;
-    static constexpr int OFF_RED = OFF_SEG + NSEG * (int)sizeof(SegDesc);
-    static constexpr int OFF_LSUM = OFF_RED + kConsumerWarps * NP * 4;
-    static constexpr int OFF_BAR = OFF_LSUM + kConsumerWarps * NP * 4;
+    static constexpr int OFF_RED = OFF_SEG + NSEG * (int)sizeof(SegDesc);   // warps' row max
+    static constexpr int OFF_LSUM = OFF_RED + kConsumerWarps * NP * 4;      // warps' row sum
+    static constexpr int OFF_ROW = OFF_LSUM + kConsumerWarps * NP * 4;      // rows' 1/L, lse
+    static constexpr int OFF_BAR = OFF_ROW + 2 * NP * 4;
     static constexpr int NBARS = 2 * NSTAGES + 2 * NSEG + 2 * kAppSlots;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int MISC_BYTES = 256;
@@ -130,6 +133,8 @@ struct DecodeCfg {
     static_assert(!FP8 || D == 128, "FP8 path is compiled for head_dim 128");
     static_assert(TILE % 1024 == 0, "tiles must keep the 1024-byte swizzle atom aligned");
     static_assert(sizeof(SegDesc) % 16 == 0, "descriptor alignment");
+    static_assert(OFF_Q % 16 == 0, "bulk copies need 16-byte aligned destinations");
+    static_assert(D != 128 || SMEM <= 113 * 1024, "two CTAs per SM at head_dim 128");
 };
 
 struct Misc {                 // CTA-wide scalars in shared memory
@@ -313,45 +318,50 @@ __device__ __forceinline__ void merge_unit(const DecodeParams &p, long long ua, 
     const long long orow =
         ((long long)s * p.q_len + head / g) * p.num_q_heads + (long long)h * g + head % g;
     auto slot_of = [&](long long c) { return 2 * c + ((ua <= c * U / G) ? 0 : 1); };
-    // pass 1: M over the pieces
-    float M = -INFINITY;
-    long long c = c_first;
-    for (; c + 3 <= c_last; c += 4) {
-        float l[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) l[i] = __ldcg(p.lse_part + slot_of(c + i) * R + head);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) M = fmaxf(M, l[i]);
-    }
-    for (; c <= c_last; ++c) M = fmaxf(M, __ldcg(p.lse_part + slot_of(c) * R + head));
-    const float Mu = M == -INFINITY ? 0.f : M;
-    // pass 2: weighted sum of the partial rows
+    // One pass over the pieces in order, NG at a time with all their loads in
+    // flight: running max M, weight sum W and weighted sum acc, rescaled
+    // whenever M grows (the online softmax merge).
+    constexpr int NG = D == 128 ? 4 : 2;
+    float M = -INFINITY, W = 0.f;
     float4 acc[MAXC];
 #pragma unroll
     for (int i = 0; i < MAXC; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    float W = 0.f;
-    auto add_piece = [&](long long cc, float w) {
-        const float4 *row = reinterpret_cast<const float4 *>(p.o_part + (slot_of(cc) * R + head) * D);
+    for (long long c = c_first; c <= c_last; c += NG) {
+        float l[NG];
+        float4 v[NG][MAXC];
 #pragma unroll
-        for (int i = 0; i < MAXC; ++i) {
-            const int col = sub + i * tph;
-            if (col < V4) {
-                const float4 v = __ldcg(row + col);
-                acc[i].x += w * v.x; acc[i].y += w * v.y; acc[i].z += w * v.z; acc[i].w += w * v.w;
+        for (int k = 0; k < NG; ++k) {
+            const bool live = c + k <= c_last;
+            const long long sl = slot_of(live ? c + k : c);
+            l[k] = live ? __ldcg(p.lse_part + sl * R + head) : -INFINITY;
+            const float4 *row = reinterpret_cast<const float4 *>(p.o_part + (sl * R + head) * D);
+#pragma unroll
+            for (int i = 0; i < MAXC; ++i) {
+                const int col = sub + i * tph;
+                v[k][i] = (live && col < V4) ? __ldcg(row + col) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
-    };
-    for (c = c_first; c + 1 <= c_last; c += 2) {
-        const float w0 = ex2(__ldcg(p.lse_part + slot_of(c) * R + head) - Mu);
-        const float w1 = ex2(__ldcg(p.lse_part + slot_of(c + 1) * R + head) - Mu);
-        W += w0 + w1;
-        add_piece(c, w0);
-        add_piece(c + 1, w1);
-    }
-    if (c <= c_last) {
-        const float w0 = ex2(__ldcg(p.lse_part + slot_of(c) * R + head) - Mu);
-        W += w0;
-        add_piece(c, w0);
+        float gm = M;
+#pragma unroll
+        for (int k = 0; k < NG; ++k) gm = fmaxf(gm, l[k]);
+        const float Mu = gm == -INFINITY ? 0.f : gm;
+        const float so = ex2(M - Mu);
+        W *= so;
+#pragma unroll
+        for (int i = 0; i < MAXC; ++i) {
+            acc[i].x *= so; acc[i].y *= so; acc[i].z *= so; acc[i].w *= so;
+        }
+#pragma unroll
+        for (int k = 0; k < NG; ++k) {
+            const float w = ex2(l[k] - Mu);
+            W += w;
+#pragma unroll
+            for (int i = 0; i < MAXC; ++i) {
+                acc[i].x += w * v[k][i].x; acc[i].y += w * v[k][i].y;
+                acc[i].z += w * v[k][i].z; acc[i].w += w * v[k][i].w;
+            }
+        }
+        M = gm;
     }
     const float inv = W > 0.f ? 1.f / W : 0.f;
 #pragma unroll
@@ -395,7 +405,9 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
     const uint32_t seg_empty = seg_full + C::NSEG * 8;
     const uint32_t app_done = seg_empty + C::NSEG * 8;
     const uint32_t app_free = app_done + kAppSlots * 8;
-    const uint32_t sP = sbase + C::OFF_P;
+    const uint32_t sO = sbase + C::OFF_O;
+    float *rowinv = reinterpret_cast<float *>(smem + C::OFF_ROW);
+    float *rowlse = rowinv + C::NP;
     const uint32_t sQ = sbase + C::OFF_Q;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -760,34 +772,45 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
 
         const float sl2 = p.scale_log2 * ksc;
 
+        // This warp's online-softmax state over its own 16 tokens of every
+        // stage: running max and (lane-partial) sum per query row, and
+        // O^T[d][row] for all D dims.  The 4 warps' states are merged once,
+        // at the end of the segment.
         float m_run[NT][2], l_run[NT][2];
-        float o_hi[C::MT][NT][4], o_lo[C::MT][NT][4];
+        float o[C::DT][NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             m_run[nt][0] = m_run[nt][1] = -INFINITY;
             l_run[nt][0] = l_run[nt][1] = 0.f;
 #pragma unroll
-            for (int mt = 0; mt < C::MT; ++mt)
+            for (int mt = 0; mt < C::DT; ++mt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) o_hi[mt][nt][e] = o_lo[mt][nt][e] = 0.f;
+                for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
         }
 
         bool abort = false;
         for (int jj = j0; jj < j1; jj += C::BPS) {
             const int nb = min(C::BPS, j1 - jj);
+            // tokens of the stage that were loaded (the stage may end with the
+            // segment or with the context)
             const int n_valid = min(ctx - jj * BS, nb * BS);
             const uint32_t slot = it % NSTAGES;
             const bool ok = mbar_wait_bounded(bar_full + 8 * slot, (it / NSTAGES) & 1);
-            if (!ok) raise_flag(p.flags, kFlagTimeout);
+            ++it;
+            if (!ok) {
+                raise_flag(p.flags, kFlagTimeout);
+                abort = true;
+                break;
+            }
             const uint32_t sK = sbase + slot * C::STAGE, sV = sK + C::STAGE_KV;
 
-            // ---- S^T = K . Q^T for this warp's 16 tokens (two MMA chains) --
-            float sacc[NT][4], sac2[NT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) sacc[nt][e] = sac2[nt][e] = 0.f;
             if (16 * warp < n_valid) {
+                // ---- S^T = K . Q^T for this warp's 16 tokens (two MMA chains)
+                float sacc[NT][4], sac2[NT][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sacc[nt][e] = sac2[nt][e] = 0.f;
                 if (!FP8) {
                     const int mi = lane >> 3;
                     const int tok = 16 * warp + (mi & 1) * 8 + (lane & 7);
@@ -826,276 +849,289 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                         }
                     }
                 }
-            }
 
-            // ---- scale, mask, stage max per head -------------------------
-            float mx[NT][2];
+                // ---- mask, this warp's max per row, weights p ----------------
+                float mx[NT][2], alpha[NT][2];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    // stage token (only the first n_valid were loaded: the
-                    // stage may end with the segment, before the context
-                    // does) and its absolute position; the row's visible
-                    // range excludes padding rows and positions past ctx
-                    const int tok = 16 * warp + gid + (e >> 1) * 8;
-                    const int pos = jj * BS + tok;
-                    const float v = sacc[nt][e] + sac2[nt][e];
-                    sacc[nt][e] = (tok < n_valid && pos >= vis_lo[nt][e & 1] &&
-                                   pos < vis_hi[nt][e & 1])
-                                      ? v * sl2 : -INFINITY;
-                }
-                mx[nt][0] = fmaxf(sacc[nt][0], sacc[nt][2]);
-                mx[nt][1] = fmaxf(sacc[nt][1], sacc[nt][3]);
-#pragma unroll
-                for (int o = 4; o < 32; o <<= 1) {
-                    mx[nt][0] = fmaxf(mx[nt][0], __shfl_xor_sync(0xffffffffu, mx[nt][0], o));
-                    mx[nt][1] = fmaxf(mx[nt][1], __shfl_xor_sync(0xffffffffu, mx[nt][1], o));
-                }
-                if (gid == 0) {
-                    red[warp * C::NP + nt * 8 + 2 * t4] = mx[nt][0];
-                    red[warp * C::NP + nt * 8 + 2 * t4 + 1] = mx[nt][1];
-                }
-            }
-            named_bar_sync(kBarConsumers, kConsumers);
-
-            // ---- new running max, probabilities to shared memory -----------
-            float alpha[NT][2];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    float sm = red[nt * 8 + 2 * t4 + e];
-#pragma unroll
-                    for (int w = 1; w < kConsumerWarps; ++w)
-                        sm = fmaxf(sm, red[w * C::NP + nt * 8 + 2 * t4 + e]);
-                    const float m_new = fmaxf(m_run[nt][e], sm);
-                    const float m_use = m_new == -INFINITY ? 0.f : m_new;
-                    alpha[nt][e] = ex2(m_run[nt][e] - m_use);
-                    m_run[nt][e] = m_new;
-                    mx[nt][e] = m_use;
-                }
-                float pr[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) pr[e] = ex2(sacc[nt][e] - mx[nt][e & 1]);
-                const int tok = 16 * warp + gid;
-                const uint32_t pa = sP + (tok * C::NP + nt * 8 + 2 * t4) * 2;
-                const uint32_t row8 = 8 * C::NP * 2;          // token + 8
-                if (!FP8) {
-                    // p = hi + lo, both bf16; the normaliser sums the fp32 p
-                    const uint32_t h0 = pack_bf16x2(pr[0], pr[1]);
-                    const uint32_t h1 = pack_bf16x2(pr[2], pr[3]);
-                    const float2 r0 = unpack_bf16x2(h0), r1 = unpack_bf16x2(h1);
-                    const uint32_t l0 = pack_bf16x2(pr[0] - r0.x, pr[1] - r0.y);
-                    const uint32_t l1 = pack_bf16x2(pr[2] - r1.x, pr[3] - r1.y);
-                    l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + pr[0] + pr[2];
-                    l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + pr[1] + pr[3];
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(pa), "r"(h0));
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(pa + row8), "r"(h1));
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(pa + C::P_BYTES), "r"(l0));
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(pa + C::P_BYTES + row8), "r"(l1));
-                } else {
-                    // f16 weights; the normaliser sums exactly the rounded values
-                    const uint32_t h0 = pack_f16x2(pr[0], pr[1]);
-                    const uint32_t h1 = pack_f16x2(pr[2], pr[3]);
-                    const float2 r0 = unpack_f16x2(h0), r1 = unpack_f16x2(h1);
-                    l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + r0.x + r1.x;
-                    l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + r0.y + r1.y;
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(pa), "r"(h0));
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(pa + row8), "r"(h1));
-                }
-            }
-            // rows past the end of the context may hold anything (NaN, Inf):
-            // zero this warp's invalid V rows so that 0 * V stays 0.
-            if (n_valid < kStageTokens) {
-                const int first = max(16 * warp, n_valid), last = 16 * warp + 16;
-                const int lines = (last - first) * C::LINES;
-                for (int i = lane >> 3; i < lines; i += 4) {
-                    const int tok = first + i / C::LINES, ln = i % C::LINES;
-                    const uint32_t a = sV + (tok / BS) * C::TILE + ln * (BS * 128) +
-                                       (tok % BS) * 128 + (lane & 7) * 16;
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0));
-                }
-                // order these generic-proxy writes before the next TMA into the slot
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            }
-            // all consumers agree on whether any of them timed out
-            abort = named_bar_sync_or(kBarConsumers, kConsumers, !ok);
-
-            // ---- O^T += V^T . P^T for this warp's D/4 dims ------------------
-#pragma unroll
-            for (int mt = 0; mt < C::MT; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+                for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        o_hi[mt][nt][e] *= alpha[nt][e & 1];
-                        o_lo[mt][nt][e] *= alpha[nt][e & 1];
+                        // stage token (only the first n_valid were loaded) and
+                        // its absolute position; the row's visible range
+                        // excludes padding rows and positions past ctx
+                        const int tok = 16 * warp + gid + (e >> 1) * 8;
+                        const int pos = jj * BS + tok;
+                        const float v = sacc[nt][e] + sac2[nt][e];
+                        sacc[nt][e] = (tok < n_valid && pos >= vis_lo[nt][e & 1] &&
+                                       pos < vis_hi[nt][e & 1])
+                                          ? v * sl2 : -INFINITY;
+                    }
+                    mx[nt][0] = fmaxf(sacc[nt][0], sacc[nt][2]);
+                    mx[nt][1] = fmaxf(sacc[nt][1], sacc[nt][3]);
+#pragma unroll
+                    for (int off = 4; off < 32; off <<= 1) {
+                        mx[nt][0] = fmaxf(mx[nt][0], __shfl_xor_sync(0xffffffffu, mx[nt][0], off));
+                        mx[nt][1] = fmaxf(mx[nt][1], __shfl_xor_sync(0xffffffffu, mx[nt][1], off));
                     }
 #pragma unroll
-            for (int kk = 0; kk < kStageTokens / 16; ++kk) {
-                if (16 * kk >= n_valid) break;
-                uint32_t pb[NT][2], pl[NT][2];
-                {
-                    const int mi = lane >> 3;
-                    const int tok = 16 * kk + 8 * (mi & 1) + (lane & 7);
-                    const uint32_t pa = NT == 1 ? sP + tok * C::NP * 2
-                                                : sP + (tok * C::NP + 8 * (mi >> 1)) * 2;
-                    if (NT == 1) {
-                        ldsm_x2_t(pa, pb[0][0], pb[0][1]);
-                        if (!FP8) ldsm_x2_t(pa + C::P_BYTES, pl[0][0], pl[0][1]);
-                    } else {
-                        ldsm_x4_t(pa, pb[0][0], pb[0][1], pb[NT - 1][0], pb[NT - 1][1]);
-                        if (!FP8)
-                            ldsm_x4_t(pa + C::P_BYTES, pl[0][0], pl[0][1], pl[NT - 1][0],
-                                      pl[NT - 1][1]);
+                    for (int e = 0; e < 2; ++e) {
+                        const float m_new = fmaxf(m_run[nt][e], mx[nt][e]);
+                        const float m_use = m_new == -INFINITY ? 0.f : m_new;
+                        alpha[nt][e] = ex2(m_run[nt][e] - m_use);
+                        m_run[nt][e] = m_new;
+                        mx[nt][e] = m_use;
                     }
                 }
+                // rows past the end of the context may hold anything (NaN,
+                // Inf): zero this warp's invalid V rows so that 0 * V stays 0
+                if (n_valid < 16 * warp + 16) {
+                    const int first = max(16 * warp, n_valid), last = 16 * warp + 16;
+                    const int lines = (last - first) * C::LINES;
+                    for (int i = lane >> 3; i < lines; i += 4) {
+                        const int tok = first + i / C::LINES, ln = i % C::LINES;
+                        const uint32_t a = sV + (tok / BS) * C::TILE + ln * (BS * 128) +
+                                           (tok % BS) * 128 + (lane & 7) * 16;
+                        sts128(a, 0u, 0u, 0u, 0u);
+                    }
+                    // order these generic-proxy writes before the next TMA
+                    // into the slot
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                }
+
+                // ---- P^T fragments (B operand, k = token, n = row) ------------
+                // The score accumulator holds S^T[token][row] in the fragment
+                // layout (lane 4r + c: tokens r and r + 8, rows 2c, 2c + 1); a
+                // warp transpose of each 8x8 half gives P^T[row][token] in
+                // the B-operand layout of the PV product.
+                uint32_t pb[NT][2], pl[NT][2];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    float pr[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) pr[e] = ex2(sacc[nt][e] - mx[nt][e & 1]);
+                    if (!FP8) {
+                        // p = hi + lo, both bf16; the normaliser sums the fp32 p
+                        const uint32_t h0 = pack_bf16x2(pr[0], pr[1]);
+                        const uint32_t h1 = pack_bf16x2(pr[2], pr[3]);
+                        const float2 q0 = unpack_bf16x2(h0), q1 = unpack_bf16x2(h1);
+                        const uint32_t l0 = pack_bf16x2(pr[0] - q0.x, pr[1] - q0.y);
+                        const uint32_t l1 = pack_bf16x2(pr[2] - q1.x, pr[3] - q1.y);
+                        l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + pr[0] + pr[2];
+                        l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + pr[1] + pr[3];
+                        pb[nt][0] = movmatrix_trans(h0);
+                        pb[nt][1] = movmatrix_trans(h1);
+                        pl[nt][0] = movmatrix_trans(l0);
+                        pl[nt][1] = movmatrix_trans(l1);
+                    } else {
+                        // f16 weights; the normaliser sums exactly the rounded values
+                        const uint32_t h0 = pack_f16x2(pr[0], pr[1]);
+                        const uint32_t h1 = pack_f16x2(pr[2], pr[3]);
+                        const float2 q0 = unpack_f16x2(h0), q1 = unpack_f16x2(h1);
+                        l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + q0.x + q1.x;
+                        l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + q0.y + q1.y;
+                        pb[nt][0] = movmatrix_trans(h0);
+                        pb[nt][1] = movmatrix_trans(h1);
+                    }
+                }
+
+                // ---- O^T += V^T . P^T over all D for this warp's tokens ------
+#pragma unroll
+                for (int mt = 0; mt < C::DT; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) o[mt][nt][e] *= alpha[nt][e & 1];
                 if (!FP8) {
                     const int mi = lane >> 3;
-                    const int tok = 16 * kk + (mi >> 1) * 8 + (lane & 7);
+                    const int tok = 16 * warp + (mi >> 1) * 8 + (lane & 7);
                     const int row = tok % BS;
                     const uint32_t rowaddr = sV + (tok / BS) * C::TILE + row * 128;
 #pragma unroll
-                    for (int mt = 0; mt < C::MT; ++mt) {
-                        const int chunk = (C::DW * warp + 16 * mt) / 8 + (mi & 1);
+                    for (int mt = 0; mt < C::DT; ++mt) {
+                        const int chunk = 2 * mt + (mi & 1);
                         const uint32_t addr = rowaddr + (chunk >> 3) * (BS * 128) +
                                               (((chunk & 7) ^ (row & 7)) << 4);
                         uint32_t a0, a1, a2, a3;
                         ldsm_x4_t(addr, a0, a1, a2, a3);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
-                            mma_bf16(o_hi[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
-                            mma_bf16(o_lo[mt][nt], a0, a1, a2, a3, pl[nt][0], pl[nt][1]);
+                            mma_bf16(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+                            mma_bf16(o[mt][nt], a0, a1, a2, a3, pl[nt][0], pl[nt][1]);
                         }
                     }
                 } else {
-                    // rows 2t, 2t+1, 2t+8, 2t+9 of this k-step; 4 bytes at
-                    // d = 32*warp + 4*gid (m-tile 0: +0,+1; m-tile 1: +2,+3)
-                    const int chunk = 2 * warp + (gid >> 2);
-                    uint32_t wv[4];
+                    // tokens 2c, 2c+1, 2c+8, 2c+9 of this warp; 16 bytes at
+                    // d = 16*gid .. 16*gid + 15 (m-tile mt: bytes 2mt, 2mt+1)
+                    uint32_t wv[4][4];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const int tok = 16 * kk + 2 * t4 + (q & 1) + (q >> 1) * 8;
+                        const int tok = 16 * warp + 2 * t4 + (q & 1) + (q >> 1) * 8;
                         const int row = tok % BS;
-                        wv[q] = lds32(sV + (tok / BS) * C::TILE + row * 128 +
-                                      ((chunk ^ (row & 7)) << 4) + 4 * (gid & 3));
+                        lds128(sV + (tok / BS) * C::TILE + row * 128 + ((gid ^ (row & 7)) << 4),
+                               wv[q][0], wv[q][1], wv[q][2], wv[q][3]);
                     }
 #pragma unroll
-                    for (int mt = 0; mt < C::MT; ++mt) {
-                        const uint32_t sel = mt == 0 ? 0x5140u : 0x7362u;
-                        const uint32_t x = prmt(wv[0], wv[1], sel);
-                        const uint32_t y = prmt(wv[2], wv[3], sel);
+                    for (int mt = 0; mt < C::DT; ++mt) {
+                        const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+                        const uint32_t x = prmt(wv[0][mt >> 1], wv[1][mt >> 1], sel);
+                        const uint32_t y = prmt(wv[2][mt >> 1], wv[3][mt >> 1], sel);
                         const uint32_t a0 = e4m3x2_to_f16x2(x & 0xffffu);
                         const uint32_t a1 = e4m3x2_to_f16x2(x >> 16);
                         const uint32_t a2 = e4m3x2_to_f16x2(y & 0xffffu);
                         const uint32_t a3 = e4m3x2_to_f16x2(y >> 16);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt)
-                            mma_f16(o_hi[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+                            mma_f16(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
                     }
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_empty + 8 * slot);
-            ++it;
-            if (abort) break;
         }
-        if (abort) return;   // uniform over the consumers; the producer drains
 
-        // ---- finish the segment ---------------------------------------------
+        // ---- finish the segment: merge the 4 warps' states -----------------
+        // In a fixed order, so that results do not depend on timing: warps 1
+        // and 3 store their O rows (buffers A and B), warps 0 and 2 add theirs
+        // to them with both weights, and the output is (A + B) / L.
+        // output dim held by accumulator element (mt, e)
+        auto dim_of = [&](int mt, int e) -> int {
+            if (!FP8) return 16 * mt + gid + (e >> 1) * 8;
+            return 16 * gid + 2 * mt + (e >> 1);
+        };
+        // A: warps 0, 1; B: warps 2, 3
+        auto store_rows = [&](int nt) {
+            float *buf = reinterpret_cast<float *>(smem + C::OFF_O + (warp >> 1) * C::OBUF);
+#pragma unroll
+            for (int mt = 0; mt < C::DT; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    buf[(2 * t4 + (e & 1)) * C::OROW + dim_of(mt, e)] = o[mt][nt][e];
+        };
+        if (warp & 1) store_rows(0);
+        // row sums over this warp's lanes; row max and sum of every warp
+        // through shared memory; all consumers agree on leaving after a timeout
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 float v = l_run[nt][e];
-                for (int o = 4; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if (gid == 0) lsum[warp * C::NP + nt * 8 + 2 * t4 + e] = v;
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                if (gid == 0) {
+                    red[warp * C::NP + nt * 8 + 2 * t4 + e] = m_run[nt][e];
+                    lsum[warp * C::NP + nt * 8 + 2 * t4 + e] = v;
+                }
             }
-        named_bar_sync(kBarConsumers, kConsumers);
-        float inv_l[NT][2], lse2[NT][2];
+        if (named_bar_sync_or(kBarConsumers, kConsumers, abort)) return;
+        // weights of this warp's and its partner's (warp + 1) O in the merged row
+        float wsc[NT][2], psc[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                float l = 0.f;
+                const int r = nt * 8 + 2 * t4 + e;
+                float M = -INFINITY;
 #pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w) l += lsum[w * C::NP + nt * 8 + 2 * t4 + e];
-                inv_l[nt][e] = l > 0.f ? vsc / l : 0.f;
-                lse2[nt][e] = l > 0.f ? m_run[nt][e] + log2f(l) : -INFINITY;
+                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[w * C::NP + r]);
+                const float Mu = M == -INFINITY ? 0.f : M;
+                wsc[nt][e] = ex2(m_run[nt][e] - Mu);
+                psc[nt][e] = ex2(red[((warp + 1) & 3) * C::NP + r] - Mu);
+                if (warp == 0 && gid == 0) {
+                    float L = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kConsumerWarps; ++w)
+                        L += lsum[w * C::NP + r] * ex2(red[w * C::NP + r] - Mu);
+                    rowinv[r] = L > 0.f ? vsc / L : 0.f;
+                    rowlse[r] = L > 0.f ? M + log2f(L) : -INFINITY;
+                }
             }
 
-        // output dim held by accumulator element (mt, e)
-        auto dim_of = [&](int mt, int e) -> int {
-            if (!FP8) return C::DW * warp + 16 * mt + gid + (e >> 1) * 8;
-            return 32 * warp + 4 * gid + 2 * mt + (e >> 1);
-        };
         // output row of query row r: query token r / g, head h*g + r % g
         auto orow = [&](int r) -> long long {
             return ((long long)s * p.q_len + r / g) * p.num_q_heads + (long long)h * g + r % g;
         };
-        if (whole) {
+        // partial results: slot 2c for the CTA's first segment, 2c+1 for its last
+        const long long pslot = 2 * cta + (useg == u0 ? 0 : 1);
+        constexpr int CPR = D / 8;   // 8-float chunks per row
 #pragma unroll
-            for (int mt = 0; mt < C::MT; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int r = nt * 8 + 2 * t4 + (e & 1);
-                        if (r < R) {
-                            const float v = (o_hi[mt][nt][e] + o_lo[mt][nt][e]) * inv_l[nt][e & 1];
-                            const long long at = orow(r) * D + dim_of(mt, e);
-                            if (p.out_f32) reinterpret_cast<float *>(p.out)[at] = v;
-                            else p.out[at] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-                        }
-                    }
-            if (p.lse_out && warp == 0 && gid == 0) {
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int r = nt * 8 + 2 * t4 + e;
-                        if (r < R) p.lse_out[orow(r)] = lse2[nt][e] * kLn2;
-                    }
+        for (int nt = 0; nt < NT; ++nt) {
+            if (nt > 0) {
+                named_bar_sync(kBarConsumers, kConsumers);   // A and B read
+                if (warp & 1) store_rows(nt);
+                named_bar_sync(kBarConsumers, kConsumers);
             }
-        } else {
-            // partial: slot 2c for the CTA's first segment, 2c+1 for its last
-            const bool first_seg = (useg == u0);
-            const long long slot = 2 * cta + (first_seg ? 0 : 1);
-            float *op = p.o_part + slot * R * D;
+            // warps 0 and 2: buffer = own O * weight + partner's O * its weight
+            if (!(warp & 1)) {
+                float *buf = reinterpret_cast<float *>(smem + C::OFF_O + (warp >> 1) * C::OBUF);
+                float part[C::DT][4];
 #pragma unroll
-            for (int mt = 0; mt < C::MT; ++mt)
+                for (int mt = 0; mt < C::DT; ++mt)
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+                    for (int e = 0; e < 4; ++e)
+                        part[mt][e] = buf[(2 * t4 + (e & 1)) * C::OROW + dim_of(mt, e)];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int r = nt * 8 + 2 * t4 + (e & 1);
-                        if (r < R)
-                            op[r * D + dim_of(mt, e)] =
-                                (o_hi[mt][nt][e] + o_lo[mt][nt][e]) * inv_l[nt][e & 1];
-                    }
-            if (warp == 0 && gid == 0) {
+                for (int mt = 0; mt < C::DT; ++mt)
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int r = nt * 8 + 2 * t4 + e;
-                        if (r < R) p.lse_part[slot * R + r] = lse2[nt][e];
-                    }
+                    for (int e = 0; e < 4; ++e)
+                        buf[(2 * t4 + (e & 1)) * C::OROW + dim_of(mt, e)] =
+                            o[mt][nt][e] * wsc[nt][e & 1] + part[mt][e] * psc[nt][e & 1];
             }
-            __threadfence();
+            named_bar_sync(kBarConsumers, kConsumers);
+            // (A + B) / L, 8 consecutive dims per step
+            for (int c = tid; c < 8 * CPR; c += kConsumers) {
+                const int rl = c / CPR, d0 = (c % CPR) * 8, r = nt * 8 + rl;
+                if (r >= R) continue;
+                const uint32_t a = sO + (rl * C::OROW + d0) * 4;
+                uint32_t x[8], y[8];
+                lds128(a, x[0], x[1], x[2], x[3]);
+                lds128(a + 16, x[4], x[5], x[6], x[7]);
+                lds128(a + C::OBUF, y[0], y[1], y[2], y[3]);
+                lds128(a + C::OBUF + 16, y[4], y[5], y[6], y[7]);
+                const float inv = rowinv[r];
+                float v[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    v[i] = (__uint_as_float(x[i]) + __uint_as_float(y[i])) * inv;
+                if (whole) {
+                    const long long at = orow(r) * D + d0;
+                    if (p.out_f32) {
+                        float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + at);
+                        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+                        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+                    } else {
+                        uint4 pk;
+                        pk.x = pack_bf16x2(v[0], v[1]);
+                        pk.y = pack_bf16x2(v[2], v[3]);
+                        pk.z = pack_bf16x2(v[4], v[5]);
+                        pk.w = pack_bf16x2(v[6], v[7]);
+                        *reinterpret_cast<uint4 *>(p.out + at) = pk;
+                    }
+                    if (p.lse_out && d0 == 0) p.lse_out[orow(r)] = rowlse[r] * kLn2;
+                } else {
+                    float4 *dst = reinterpret_cast<float4 *>(p.o_part + (pslot * R + r) * D + d0);
+                    dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+                    dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+                    if (d0 == 0) p.lse_part[pslot * R + r] = rowlse[r];
+                }
+            }
+        }
+        if (!whole) {
+            // every consumer's partial stores precede the barrier; the arrival
+            // count is an acquire-release atomic, so the last CTA to arrive
+            // sees all pieces (the barriers carry the ordering to the other
+            // threads of both CTAs)
             named_bar_sync(kBarConsumers, kConsumers);
             // unit tile range [ua, ub) in work space and the CTAs that share it
             const long long ua = useg - (j0 - jlo);
             const long long ub = ua + (nunit - jlo);
             const long long c_first = cta_of(ua, U, G), c_last = cta_of(ub - 1, U, G);
             if (tid == 0) {
-                const int prev = atomicAdd(p.counters + (long long)s * Hkv + h, 1);
+                const int prev = atom_add_acq_rel_gpu(p.counters + (long long)s * Hkv + h, 1);
                 misc->is_last = (prev == (int)(c_last - c_first));
             }
             named_bar_sync(kBarConsumers, kConsumers);
             if (misc->is_last) {
-                __threadfence();
                 merge_unit<D>(p, ua, U, G, c_first, c_last, s, h);
                 if (tid == 0) p.counters[(long long)s * Hkv + h] = 0;
             }
