@@ -142,8 +142,9 @@ struct Misc {                 // CTA-wide scalars in shared memory
     int s0;
     int is_last;
     int found;
-    int pad;
+    int win_ok;               // win holds the context lengths of s0 .. s0 + 31
     long long warp_tmp[8];
+    int win[32];
 };
 
 // ------------------------------------------------------------------ helpers
@@ -260,11 +261,16 @@ __device__ __forceinline__ void next_unit(Cursor &c, const DecodeParams &p) {
 
 template <int BS>
 __device__ __forceinline__ Cursor first_unit(const DecodeParams &p, int s0, long long pfx0,
-                                            long long u0) {
+                                            long long u0, const int *win) {
     Cursor c;
     c.s = s0;
-    c.wbase = -64;                   // empty window: the first read loads it
-    c.wval = 0;
+    if (win) {                       // the prologue's copy of s0 .. s0 + 31
+        c.wbase = s0;
+        c.wval = win[threadIdx.x & 31];
+    } else {
+        c.wbase = -64;               // empty window: the first read loads it
+        c.wval = 0;
+    }
     set_seq<BS>(c, p);
     c.h = (int)((u0 - pfx0) / c.w);
     c.a = pfx0 + (long long)c.h * c.w;
@@ -390,6 +396,7 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
 paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
     using C = DecodeCfg<D, BS, NT, FP8, NSTAGES>;
+    static_assert(sizeof(Misc) <= C::MISC_BYTES, "CTA scalars");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -441,36 +448,75 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         tma_prefetch_desc(&tmV);
     }
 
-    // ---- prologue: total tiles and this CTA's range --------------------
-    long long mine = 0;
-    for (int s = tid; s < B; s += kThreads) mine += seq_weight<BS>(p, s);
-    const long long U = block_sum(mine, misc) * Hkv;
-    // CTAs beyond the tile count get no range, so every range is non-empty
+    // units with an empty context: out = 0, lse = -inf for all their query
+    // rows; thread t of nt per CTA, CTA c of nc
+    auto zero_fill = [&](int t, int nt, long long nc) {
+        for (long long v = cta + nc * t; v < (long long)B * Hkv; v += nc * nt) {
+            const int s = (int)(v / Hkv), h = (int)(v % Hkv);
+            if (ctx_of<BS>(p, s) != 0) continue;
+            for (int i = 0; i < p.q_len; ++i) {
+                const long long row0 =
+                    ((long long)s * p.q_len + i) * p.num_q_heads + (long long)h * g;
+                const int words = p.out_f32 ? 2 * g * D : g * D;   // 16-bit words
+                uint16_t *o = p.out + row0 * D * (p.out_f32 ? 2 : 1);
+                for (int e = 0; e < words; ++e) o[e] = 0;
+                if (p.lse_out)
+                    for (int e = 0; e < g; ++e) p.lse_out[row0 + e] = -INFINITY;
+            }
+        }
+    };
+
+    // ---- prologue: total work and this CTA's range --------------------
+    // Thread t reads the context lengths of sequences t*KS .. t*KS + KS - 1
+    // of the first CH once and keeps them; one block scan gives every
+    // sequence's work prefix.  Longer batches are summed in further passes.
+    constexpr int KS = 4, CH = KS * kThreads;
+    int cl[KS];
+    long long wk[KS], tsum = 0;
+#pragma unroll
+    for (int k = 0; k < KS; ++k) {
+        const int s = tid * KS + k;
+        cl[k] = s < B ? ctx_of<BS>(p, s) : 0;
+        wk[k] = s < B ? unit_weight(nblk_of<BS>(cl[k]) - first_block<BS>(cl[k], p), p.unit_cost)
+                      : 0;
+        tsum += wk[k];
+    }
+    long long W0;                                   // one KV head's work in the first CH
+    const long long excl0 = block_scan(tsum, W0, misc) - tsum;
+    long long U1 = W0;                              // one KV head's work in the batch
+    for (int base = CH; base < B; base += kThreads) {
+        const int s = base + tid;
+        U1 += block_sum(s < B ? seq_weight<BS>(p, s) : 0, misc);
+    }
+    const long long U = U1 * Hkv;
+    // CTAs beyond the work count get no range, so every range is non-empty
     const long long G = min((long long)gridDim.x, U);
     const long long u0 = cta < G ? cta * U / G : 0, u1 = cta < G ? (cta + 1) * U / G : 0;
-
-    // units with an empty context: out = 0, lse = -inf for all their query
-    // rows (each thread checks its own units, spread over all CTAs)
-    for (long long v = cta + (long long)gridDim.x * tid; v < (long long)B * Hkv;
-         v += (long long)gridDim.x * kThreads) {
-        const int s = (int)(v / Hkv), h = (int)(v % Hkv);
-        if (ctx_of<BS>(p, s) != 0) continue;
-        for (int i = 0; i < p.q_len; ++i) {
-            const long long row0 =
-                ((long long)s * p.q_len + i) * p.num_q_heads + (long long)h * g;
-            const int words = p.out_f32 ? 2 * g * D : g * D;   // 16-bit words
-            uint16_t *o = p.out + row0 * D * (p.out_f32 ? 2 : 1);
-            for (int e = 0; e < words; ++e) o[e] = 0;
-            if (p.lse_out)
-                for (int e = 0; e < g; ++e) p.lse_out[row0 + e] = -INFINITY;
-        }
+    if (U == 0) {             // every context is empty
+        zero_fill(tid, kThreads, gridDim.x);
+        return;
     }
     if (u0 >= u1) return;   // nothing in flight, no barrier shared past this point
 
-    // locate the sequence that holds tile u0
+    // locate the sequence that holds work index u0
     {
-        long long base = 0;
-        for (int sb = 0; sb < B; sb += kThreads) {
+        long long a = excl0 * Hkv;
+#pragma unroll
+        for (int k = 0; k < KS; ++k) {
+            const int s = tid * KS + k;
+            const long long w = wk[k] * Hkv;
+            if (s < B && w > 0 && a <= u0 && u0 < a + w) {
+                misc->s0 = s;
+                misc->pfx0 = a;
+                misc->found = 1;
+            }
+            a += w;
+        }
+    }
+    __syncthreads();
+    if (!misc->found) {       // u0 lies past the first CH sequences
+        long long base = W0 * Hkv;
+        for (int sb = CH; sb < B; sb += kThreads) {
             const int s = sb + tid;
             const long long wgt = s < B ? seq_weight<BS>(p, s) * Hkv : 0;
             long long tot;
@@ -486,7 +532,18 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             if (misc->found) break;
         }
     }
+    // context lengths of s0 .. s0 + 31 for the walkers' first window
+    {
+        const int s0 = misc->s0;
+#pragma unroll
+        for (int k = 0; k < KS; ++k) {
+            const int s = tid * KS + k;
+            if (s >= s0 && s < s0 + 32) misc->win[s - s0] = cl[k];
+        }
+        if (tid == 0) misc->win_ok = (s0 + 32 <= CH || B <= CH) ? 1 : 0;
+    }
     __syncthreads();
+    const int *win0 = misc->win_ok ? misc->win : nullptr;
 
     if (warp == kConsumerWarps + 1) {
         // ================= appender warp (fused append only) ===============
@@ -496,8 +553,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         // before async-proxy reads, and signals the producer, which waits for
         // the signal before loading that block.  Only this CTA reads the
         // unit's last tile, so no other CTA can see the row half-written.
+        // First it writes the empty units (spread over the G CTAs that have work).
+        zero_fill(lane, 32, G);
         if (p.k_new == nullptr) return;
-        Cursor cur = first_unit<BS>(p, misc->s0, misc->pfx0, u0);
+        Cursor cur = first_unit<BS>(p, misc->s0, misc->pfx0, u0, win0);
         uint32_t ait = 0;
         for (; cur.a < u1; next_unit<BS>(cur, p)) {
             const long long r0 = max(0LL, u0 - cur.a);
@@ -539,7 +598,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
 
     if (warp == kConsumerWarps) {
         // ================= producer warp ====================================
-        Cursor cur = first_unit<BS>(p, misc->s0, misc->pfx0, u0);
+        Cursor cur = first_unit<BS>(p, misc->s0, misc->pfx0, u0, win0);
         const uint32_t qtok = (uint32_t)(g * D * 2);          // one query token's rows
         uint32_t it = 0, sit = 0, ait = 0;
         bool ok = true;
