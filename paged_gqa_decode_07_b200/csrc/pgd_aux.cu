@@ -114,6 +114,10 @@ __global__ void __launch_bounds__(128)
 merge_partials_kernel(const float *__restrict__ o_part, const float *__restrict__ lse_part,
                       int32_t parts, int32_t rows, int32_t head_dim, uint16_t *out,
                       float *lse_out) {
+    // programmatic dependent launch: the split results come from the
+    // previous launch on the stream
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int r = blockIdx.x;
     constexpr float kLog2e = 1.4426950408889634f;
     float M = -INFINITY;
@@ -136,9 +140,17 @@ merge_partials_kernel(const float *__restrict__ o_part, const float *__restrict_
 cudaError_t launch_merge_partials(const float *o_part, const float *lse_part, int32_t parts,
                                   int32_t rows, int32_t head_dim, uint16_t *out, float *lse_out,
                                   cudaStream_t stream) {
-    merge_partials_kernel<<<rows, 128, 0, stream>>>(o_part, lse_part, parts, rows, head_dim, out,
-                                                    lse_out);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(rows));
+    cfg.blockDim = dim3(128);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, merge_partials_kernel, o_part, lse_part, parts, rows, head_dim,
+                              out, lse_out);
 }
 
 }  // namespace pgd

@@ -43,20 +43,29 @@ def _world(group) -> int:
     return dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1
 
 
+def _rank(group) -> int:
+    return dist.get_rank(group) if dist.is_available() and dist.is_initialized() else 0
+
+
 def gather_partials(o_part: torch.Tensor, lse_part: torch.Tensor, o_all: torch.Tensor,
                     lse_all: torch.Tensor, group=None) -> None:
     """All-gather every rank's split result: o_part [rows][D] (any shape with
     rows * D elements) and lse_part [rows] into o_all [W][rows][D] and
-    lse_all [W][rows], rank r at index r."""
-    W = _world(group)
+    lse_all [W][rows], rank r at index r.  o_part / lse_part may already be
+    this rank's slots of o_all / lse_all (then nothing is copied locally)."""
+    W, r = _world(group), _rank(group)
     if o_all.shape[0] != W or lse_all.shape[0] != W:
         raise ValueError("gather buffers must have one slot per rank")
-    if W == 1:
-        o_all[0].view(-1).copy_(o_part.reshape(-1))
-        lse_all[0].view(-1).copy_(lse_part.reshape(-1))
-        return
-    dist.all_gather_into_tensor(o_all.view(-1), o_part.reshape(-1), group=group)
-    dist.all_gather_into_tensor(lse_all.view(-1), lse_part.reshape(-1), group=group)
+    for part, full in ((o_part, o_all), (lse_part, lse_all)):
+        in_place = part.data_ptr() == full[r].data_ptr()
+        if W == 1:
+            if not in_place:
+                full[0].view(-1).copy_(part.reshape(-1))
+            continue
+        src = part.reshape(-1)
+        if in_place and dist.get_backend(group) != "nccl":
+            src = src.clone()          # only NCCL gathers in place
+        dist.all_gather_into_tensor(full.view(-1), src, group=group)
 
 
 class KVPDecoder:
@@ -75,10 +84,12 @@ class KVPDecoder:
         dev = torch.device("cuda") if device is None else torch.device(device)
         rows = num_seqs * num_q_heads
         f32 = dict(dtype=torch.float32, device=dev)
-        self.o_local = torch.empty((num_seqs, num_q_heads, head_dim), **f32)
-        self.lse_local = torch.empty((num_seqs, num_q_heads), **f32)
         self.o_all = torch.empty((self.world, rows, head_dim), **f32)
         self.lse_all = torch.empty((self.world, rows), **f32)
+        # this rank's split result is decoded straight into its gather slot
+        r = _rank(group)
+        self.o_local = self.o_all[r].view(num_seqs, num_q_heads, head_dim)
+        self.lse_local = self.lse_all[r].view(num_seqs, num_q_heads)
         self.out = torch.empty((num_seqs, num_q_heads, head_dim), dtype=torch.bfloat16,
                                device=dev)
         self.lse = torch.empty((rows,), **f32)

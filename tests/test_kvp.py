@@ -96,13 +96,20 @@ def _kvp_worker(rank, world, port, q):
         o_all = torch.empty((world, rows, w.head_dim), dtype=torch.float64)
         lse_all = torch.empty((world, rows), dtype=torch.float64)
         K.gather_partials(torch.from_numpy(o), torch.from_numpy(lse), o_all, lse_all)
+        # the same exchange with each rank's result already in its own slot
+        o_in = torch.zeros_like(o_all)
+        lse_in = torch.zeros_like(lse_all)
+        o_in[rank].copy_(torch.from_numpy(o).reshape(rows, -1))
+        lse_in[rank].copy_(torch.from_numpy(lse).reshape(-1))
+        K.gather_partials(o_in[rank], lse_in[rank], o_in, lse_in)
+        same = bool(torch.equal(o_in, o_all) and torch.equal(lse_in, lse_all))
         merged, mlse = oracle.merge_partials(o_all.numpy(), lse_all.numpy())
         ref, rlse = oracle.paged_decode(w.q, w.k_cache, w.v_cache, w.block_table,
                                         w.context_lens, w.num_kv_heads, w.scale)
         err = float(np.max(np.abs(merged - ref.reshape(rows, -1))))
         live = np.isfinite(rlse.reshape(-1))
         lerr = float(np.max(np.abs(mlse[live] - rlse.reshape(-1)[live])))
-        dead_ok = bool(np.all(np.isneginf(mlse[~live])) and np.all(merged[~live] == 0))
+        dead_ok = same and bool(np.all(np.isneginf(mlse[~live])) and np.all(merged[~live] == 0))
         q.put((rank, err, lerr, dead_ok))
     finally:
         dist.destroy_process_group()
