@@ -20,6 +20,8 @@ Other rows of the path, same JSON line, each on its own workload shape:
                            among them) and/or a sliding window of W tokens
                            (pgd_paged_decode_attention_ex); the bytes count
                            the visible K/V rows only
+    --math cuda_core       the decode kernel's q.k and p.V as FP32 FMAs with
+                           warp-shuffle sums instead of mma.sync (comparison)
     --kvp                  one batch with every sequence's KV split along its
                            length over the N ranks: slice decode to fp32,
                            all-gather, log-sum-exp merge (strong scaling)
@@ -369,6 +371,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.current_stream()
+    pgd.set_decode_math(args.math)
     if args.kvp:
         # one batch split over the ranks: the same data on every rank
         w = make_workload(args.workload, seed=0, shape_seed=0)
@@ -476,6 +479,8 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0:
         cfg = workload_desc(w)
         cfg.update(m.cfg)
+        if args.math != "tensor_core":
+            cfg["math"] = args.math
         kv_mb = w.algorithmic_bytes(max(1, args.q_len), args.window)["kv"] / 1e6
         cfg.update({"parallelism": (f"KV parallel over {world} rank(s) (one batch, each "
                                     f"sequence split along its length)") if args.kvp else
@@ -632,6 +637,9 @@ def main():
                     help="query tokens per sequence (causal among them)")
     ap.add_argument("--window", type=int, default=0,
                     help="sliding window in tokens (0 = whole context)")
+    ap.add_argument("--math", choices=["tensor_core", "cuda_core"], default="tensor_core",
+                    help="consumer math of the decode kernel (cuda_core: FMA + warp shuffles, "
+                         "bf16 head_dim 128 with <= 8 query rows per KV head)")
     ap.add_argument("--kvp", action="store_true",
                     help="split every sequence's KV over the ranks (strong scaling)")
     args = ap.parse_args()

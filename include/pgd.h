@@ -268,6 +268,32 @@ pgd_status pgd_paged_decode_attention_ex(
     void *workspace, size_t workspace_bytes, int32_t num_ctas, void *stream);
 
 /* ------------------------------------------------------------------------ */
+/* Consumer math of the decode kernels                                      */
+/* ------------------------------------------------------------------------ */
+/*
+ * The decode kernels form q.k and p.V on the tensor cores by default: a small
+ * mma.sync per 16 tokens with the group's query rows on the narrow side.
+ * PGD_MATH_CUDA_CORE selects a variant that does the same arithmetic with
+ * FP32 FMAs and warp-shuffle reductions (the form the decode kernels of the
+ * "attention kernels" page describe), kept so that the two can be measured
+ * against each other on this bandwidth-bound path.  It covers bf16 caches
+ * with head_dim 128 and at most 8 query rows per KV head (g * q_len <= 8);
+ * while it is selected, other shapes return PGD_ERR_UNSUPPORTED.  Results of
+ * the two agree within the stated tolerances, not bit for bit.
+ *
+ * pgd_set_decode_math -- process-wide setting for every decode entry point
+ * that follows (host only; PGD_ERR_INVALID_ARG for an unknown value).
+ * pgd_get_decode_math -- the current setting.
+ */
+typedef enum {
+    PGD_MATH_TENSOR_CORE = 0,
+    PGD_MATH_CUDA_CORE = 1
+} pgd_decode_math;
+
+pgd_status pgd_set_decode_math(pgd_decode_math math);
+pgd_decode_math pgd_get_decode_math(void);
+
+/* ------------------------------------------------------------------------ */
 /* KV parallelism: one sequence's KV split along its length over GPUs       */
 /* ------------------------------------------------------------------------ */
 /*

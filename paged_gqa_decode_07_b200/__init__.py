@@ -8,11 +8,13 @@ from ._binding import (  # noqa: F401
     PGD_KV_BF16, PGD_KV_FP8_E4M3, PGDError, LIB_PATH, lib_path, load_library, kv_append,
     kv_append_quant, paged_decode_attention, paged_decode_attention_ex,
     paged_decode_attention_noalloc, paged_decode_partial, kvp_plan, decode_step,
-    merge_partials, decode_workspace_bytes, get_device_error, shutdown,
+    merge_partials, decode_workspace_bytes, get_device_error, shutdown, set_decode_math,
+    get_decode_math,
 )
 from . import kvp  # noqa: F401,E402
 
 __all__ = ["kv_append", "kv_append_quant", "paged_decode_attention", "paged_decode_attention_ex",
            "paged_decode_attention_noalloc", "paged_decode_partial", "kvp_plan", "decode_step",
            "merge_partials", "decode_workspace_bytes", "get_device_error", "shutdown",
-           "PGDError", "load_library", "lib_path", "kvp", "PGD_KV_BF16", "PGD_KV_FP8_E4M3"]
+           "set_decode_math", "get_decode_math", "PGDError", "load_library", "lib_path", "kvp",
+           "PGD_KV_BF16", "PGD_KV_FP8_E4M3"]

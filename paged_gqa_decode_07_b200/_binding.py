@@ -68,6 +68,10 @@ def load_library():
     lib.pgd_paged_decode_partial.restype = st
     lib.pgd_paged_decode_partial.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32, i32,
                                              i32, f32, st, P, P, P, P, P, sz, i32, P]
+    lib.pgd_set_decode_math.restype = st
+    lib.pgd_set_decode_math.argtypes = [st]
+    lib.pgd_get_decode_math.restype = st
+    lib.pgd_get_decode_math.argtypes = []
     lib.pgd_kvp_plan.restype = st
     lib.pgd_kvp_plan.argtypes = [P, i32, i32, i32, i32, P, P]
     lib.pgd_decode_step.restype = st
@@ -315,6 +319,23 @@ def paged_decode_partial(q, k_cache, v_cache, block_table, context_lens, num_q_h
         _ptr(o_part), _ptr(lse_part), _ptr(workspace), ws_bytes, int(num_ctas), _stream(stream)),
         "pgd_paged_decode_partial")
     return o_part, lse_part
+
+
+_MATH = {"tensor_core": 0, "cuda_core": 1}
+
+
+def set_decode_math(math: str) -> None:
+    """Consumer math of the decode kernels, process-wide (pgd_set_decode_math):
+    "tensor_core" (default) or "cuda_core" (FMA + warp shuffles; bf16,
+    head_dim 128, at most 8 query rows per KV head)."""
+    if math not in _MATH:
+        raise ValueError(f"math must be one of {sorted(_MATH)}")
+    _check(load_library().pgd_set_decode_math(_MATH[math]), "pgd_set_decode_math")
+
+
+def get_decode_math() -> str:
+    v = int(load_library().pgd_get_decode_math())
+    return {b: a for a, b in _MATH.items()}[v]
 
 
 def kvp_plan(context_lens, block_size: int, world_size: int, rank: int):

@@ -22,7 +22,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpgd.so")
 
 SOURCES = ["pgd_api.cu", "pgd_aux.cu", "pgd_decode_bf16_d128.cu", "pgd_decode_bf16_d256.cu",
-           "pgd_decode_fp8_d128.cu"]
+           "pgd_decode_fp8_d128.cu", "pgd_decode_bf16_d128_cc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-I" + INCLUDE,
          "-I" + CSRC, "--expt-relaxed-constexpr"]

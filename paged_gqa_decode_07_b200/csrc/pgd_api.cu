@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstring>
@@ -159,7 +160,23 @@ bool pick_bs(int bs, int nt, Variant *v) {
     return false;
 }
 
-bool pick_variant(int D, int bs, int nt, bool fp8, Variant *v) {
+// Consumer math of the decode kernels (pgd_set_decode_math); process-wide.
+std::atomic<int> g_math{PGD_MATH_TENSOR_CORE};
+
+template <int CC>
+bool pick_cuda_core(int bs, Variant *v) {
+    if (bs == 16) *v = {&launch_decode<128, 16, 1, false, CC>, &decode_ctas_per_sm<128, 16, 1, false, CC>};
+    else if (bs == 32) *v = {&launch_decode<128, 32, 1, false, CC>, &decode_ctas_per_sm<128, 32, 1, false, CC>};
+    else if (bs == 64) *v = {&launch_decode<128, 64, 1, false, CC>, &decode_ctas_per_sm<128, 64, 1, false, CC>};
+    else return false;
+    return true;
+}
+
+bool pick_variant(int D, int bs, int nt, bool fp8, int rows, Variant *v) {
+    if (g_math.load() == PGD_MATH_CUDA_CORE) {
+        if (fp8 || D != 128 || rows > 8) return false;
+        return rows <= 4 ? pick_cuda_core<4>(bs, v) : pick_cuda_core<8>(bs, v);
+    }
     if (!fp8 && D == 128) return pick_bs<128, false>(bs, nt, v);
     if (!fp8 && D == 256) return pick_bs<256, false>(bs, nt, v);
     if (fp8 && D == 128) return pick_bs<128, true>(bs, nt, v);
@@ -312,7 +329,7 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     if (st != PGD_OK) return st;
     const int nt = rows > 8 ? 2 : 1;
     Variant var;
-    if (!pick_variant(head_dim, block_size, nt, fp8, &var)) return PGD_ERR_UNSUPPORTED;
+    if (!pick_variant(head_dim, block_size, nt, fp8, rows, &var)) return PGD_ERR_UNSUPPORTED;
 
     // ---- grid: a full wave of resident CTAs, fewer for small batches ---------
     long long grid = num_ctas;
@@ -456,6 +473,16 @@ pgd_status pgd_paged_decode_partial(
                        block_size, num_blocks, scale, kv_dtype, k_scale, v_scale, nullptr,
                        nullptr, o_part, lse_part, workspace, workspace_bytes, num_ctas, stream,
                        1, 0, true);
+}
+
+pgd_status pgd_set_decode_math(pgd_decode_math math) {
+    if (math != PGD_MATH_TENSOR_CORE && math != PGD_MATH_CUDA_CORE) return PGD_ERR_INVALID_ARG;
+    g_math.store(math);
+    return PGD_OK;
+}
+
+pgd_decode_math pgd_get_decode_math(void) {
+    return static_cast<pgd_decode_math>(g_math.load());
 }
 
 pgd_status pgd_kvp_plan(const int32_t *context_lens, int32_t num_seqs, int32_t block_size,
@@ -644,7 +671,7 @@ extern "C" pgd_status pgd_paged_decode_attention_noalloc(
     if ((st = static_scratch(&scratch)) != PGD_OK) return st;
     const int nt = g > 8 ? 2 : 1;
     Variant var;
-    if (!pick_variant(head_dim, block_size, nt, fp8, &var)) return PGD_ERR_UNSUPPORTED;
+    if (!pick_variant(head_dim, block_size, nt, fp8, g, &var)) return PGD_ERR_UNSUPPORTED;
 
     // grid: as the allocating entry point, then capped so that the split
     // partials fit behind the counters in the static array

@@ -98,7 +98,10 @@ struct SegDesc {
     int jlo;          // first block any query row of the unit sees
 };
 
-template <int D, int BS, int NT, bool FP8, int NSTAGES>
+// CC = 0: tensor-core (mma.sync) consumers; CC = 4 or 8: the CUDA-core
+// variant (FMA dot products with warp-shuffle reductions) for up to CC query
+// rows, kept to compare the two on this bandwidth-bound path.
+template <int D, int BS, int NT, bool FP8, int NSTAGES, int CC = 0>
 struct DecodeCfg {
     static constexpr int E = FP8 ? 1 : 2;                // bytes per KV element
     static constexpr int ROW = D * E;                    // bytes per K/V row
@@ -113,7 +116,7 @@ struct DecodeCfg {
     static constexpr int QSLOT = NP * D * 2;             // query rows of one unit
     // descriptor ring depth (one slot for 16 query rows at head_dim 128, so
     // that two CTAs still fit on an SM)
-    static constexpr int NSEG = D == 128 ? (QSLOT >= 4096 ? 1 : 3) : 2;
+    static constexpr int NSEG = CC ? 2 : (D == 128 ? (QSLOT >= 4096 ? 1 : 3) : 2);
     static constexpr int OROW = D + 4;                   // sO row stride in floats
     // shared memory carve-up (offsets from a 1024-aligned base)
     static constexpr int OFF_O = NSTAGES * STAGE;        // two 8-row O buffers
@@ -123,7 +126,11 @@ struct DecodeCfg {
     static constexpr int OFF_RED = OFF_SEG + NSEG * (int)sizeof(SegDesc);   // warps' row max
     static constexpr int OFF_LSUM = OFF_RED + kConsumerWarps * NP * 4;      // warps' row sum
     static constexpr int OFF_ROW = OFF_LSUM + kConsumerWarps * NP * 4;      // rows' 1/L, lse
-    static constexpr int OFF_BAR = OFF_ROW + 2 * NP * 4;
+    // CUDA-core variant: each warp's softmax weights of a stage [16][CC] and
+    // the rows' rescale factors [CC]
+    static constexpr int PWF = 16 * 8 + 8;                // floats per warp
+    static constexpr int OFF_PW = OFF_ROW + 2 * NP * 4;
+    static constexpr int OFF_BAR = OFF_PW + (CC ? kConsumerWarps * PWF * 4 : 0);
     static constexpr int NBARS = 2 * NSTAGES + 2 * NSEG + 2 * kAppSlots;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int MISC_BYTES = 256;
@@ -391,11 +398,13 @@ __device__ __forceinline__ void merge_unit(const DecodeParams &p, long long ua, 
 }
 
 // ------------------------------------------------------------------ kernel
-template <int D, int BS, int NT, bool FP8, int NSTAGES>
+template <int D, int BS, int NT, bool FP8, int NSTAGES, int CC = 0>
 __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
 paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
-    using C = DecodeCfg<D, BS, NT, FP8, NSTAGES>;
+    using C = DecodeCfg<D, BS, NT, FP8, NSTAGES, CC>;
+    static_assert(CC == 0 || (D == 128 && !FP8 && NT == 1 && (CC == 4 || CC == 8)),
+                  "CUDA-core variant: bf16, head_dim 128, 4 or 8 rows");
     static_assert(sizeof(Misc) <= C::MISC_BYTES, "CTA scalars");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -788,324 +797,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         const bool whole = (j0 == jlo && j1 == nunit);
         const int R = p.rows;
 
-        // visible token range [lo, hi) of the two query rows this lane holds
-        // per n-tile (rows 8*nt + 2*t4 + {0, 1}; row = query token * g + head)
-        int vis_lo[NT][2], vis_hi[NT][2];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int row = nt * 8 + 2 * t4 + e;
-                const int hi = ctx - p.q_len + 1 + row / g;
-                vis_hi[nt][e] = row < R ? hi : 0;
-                vis_lo[nt][e] = (row < R && p.window > 0) ? max(0, hi - p.window) : 0;
-            }
-
-        // query fragments (B operand, Q^T[d][row]) from the slot
-        uint32_t qf[C::KSTEPS][NT][2];
-        {
-            const uint32_t qb = sQ + qs * C::QSLOT;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int head = nt * 8 + gid;      // query row held as B column
-                const bool live = head < R;
-                const uint32_t qr = qb + (live ? head : 0) * D * 2;
-#pragma unroll
-                for (int k = 0; k < C::KSTEPS; ++k) {
-                    uint32_t b0, b1;
-                    if (!FP8) {   // k index 2t, 2t+1 | 2t+8, 2t+9  <->  same d
-                        b0 = lds32(qr + (16 * k + 2 * t4) * 2);
-                        b1 = lds32(qr + (16 * k + 8 + 2 * t4) * 2);
-                    } else {      // k index permuted to d = 16k + 4t + {0,1 | 2,3}
-                        b0 = bf16x2_to_f16x2(lds32(qr + (16 * k + 4 * t4) * 2));
-                        b1 = bf16x2_to_f16x2(lds32(qr + (16 * k + 4 * t4 + 2) * 2));
-                    }
-                    qf[k][nt][0] = live ? b0 : 0u;
-                    qf[k][nt][1] = live ? b1 : 0u;
-                }
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(seg_empty + 8 * qs);   // the slot may be refilled
-        ++sit;
-
         const float sl2 = p.scale_log2 * ksc;
-
-        // This warp's online-softmax state over its own 16 tokens of every
-        // stage: running max and (lane-partial) sum per query row, and
-        // O^T[d][row] for all D dims.  The 4 warps' states are merged once,
-        // at the end of the segment.
-        float m_run[NT][2], l_run[NT][2];
-        float o[C::DT][NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            m_run[nt][0] = m_run[nt][1] = -INFINITY;
-            l_run[nt][0] = l_run[nt][1] = 0.f;
-#pragma unroll
-            for (int mt = 0; mt < C::DT; ++mt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
-        }
-
-        bool abort = false;
-        for (int jj = j0; jj < j1; jj += C::BPS) {
-            const int nb = min(C::BPS, j1 - jj);
-            // tokens of the stage that were loaded (the stage may end with the
-            // segment or with the context)
-            const int n_valid = min(ctx - jj * BS, nb * BS);
-            const uint32_t slot = it % NSTAGES;
-            const bool ok = mbar_wait_bounded(bar_full + 8 * slot, (it / NSTAGES) & 1);
-            ++it;
-            if (!ok) {
-                raise_flag(p.flags, kFlagTimeout);
-                abort = true;
-                break;
-            }
-            const uint32_t sK = sbase + slot * C::STAGE, sV = sK + C::STAGE_KV;
-
-            if (16 * warp < n_valid) {
-                // ---- S^T = K . Q^T for this warp's 16 tokens (two MMA chains)
-                float sacc[NT][4], sac2[NT][4];
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) sacc[nt][e] = sac2[nt][e] = 0.f;
-                if (!FP8) {
-                    const int mi = lane >> 3;
-                    const int tok = 16 * warp + (mi & 1) * 8 + (lane & 7);
-                    const int row = tok % BS;
-                    const uint32_t rowaddr = sK + (tok / BS) * C::TILE + row * 128;
-#pragma unroll
-                    for (int k = 0; k < C::KSTEPS; ++k) {
-                        const int chunk = 2 * k + (mi >> 1);
-                        const uint32_t addr = rowaddr + (chunk >> 3) * (BS * 128) +
-                                              (((chunk & 7) ^ (row & 7)) << 4);
-                        uint32_t a0, a1, a2, a3;
-                        ldsm_x4(addr, a0, a1, a2, a3);
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            if (k & 1) mma_bf16(sac2[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
-                            else       mma_bf16(sacc[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
-                        }
-                    }
-                } else {
-                    const int tok0 = 16 * warp + gid, tok1 = tok0 + 8;
-                    const int r0 = tok0 % BS, r1 = tok1 % BS;
-                    const uint32_t base0 = sK + (tok0 / BS) * C::TILE + r0 * 128 + 4 * t4;
-                    const uint32_t base1 = sK + (tok1 / BS) * C::TILE + r1 * 128 + 4 * t4;
-#pragma unroll
-                    for (int k = 0; k < C::KSTEPS; ++k) {
-                        const uint32_t w0 = lds32(base0 + ((k ^ (r0 & 7)) << 4));
-                        const uint32_t w1 = lds32(base1 + ((k ^ (r1 & 7)) << 4));
-                        const uint32_t a0 = e4m3x2_to_f16x2(w0 & 0xffffu);
-                        const uint32_t a2 = e4m3x2_to_f16x2(w0 >> 16);
-                        const uint32_t a1 = e4m3x2_to_f16x2(w1 & 0xffffu);
-                        const uint32_t a3 = e4m3x2_to_f16x2(w1 >> 16);
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            if (k & 1) mma_f16(sac2[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
-                            else       mma_f16(sacc[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
-                        }
-                    }
-                }
-
-                // ---- mask, this warp's max per row, weights p ----------------
-                float mx[NT][2], alpha[NT][2];
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        // stage token (only the first n_valid were loaded) and
-                        // its absolute position; the row's visible range
-                        // excludes padding rows and positions past ctx
-                        const int tok = 16 * warp + gid + (e >> 1) * 8;
-                        const int pos = jj * BS + tok;
-                        const float v = sacc[nt][e] + sac2[nt][e];
-                        sacc[nt][e] = (tok < n_valid && pos >= vis_lo[nt][e & 1] &&
-                                       pos < vis_hi[nt][e & 1])
-                                          ? v * sl2 : -INFINITY;
-                    }
-                    mx[nt][0] = fmaxf(sacc[nt][0], sacc[nt][2]);
-                    mx[nt][1] = fmaxf(sacc[nt][1], sacc[nt][3]);
-#pragma unroll
-                    for (int off = 4; off < 32; off <<= 1) {
-                        mx[nt][0] = fmaxf(mx[nt][0], __shfl_xor_sync(0xffffffffu, mx[nt][0], off));
-                        mx[nt][1] = fmaxf(mx[nt][1], __shfl_xor_sync(0xffffffffu, mx[nt][1], off));
-                    }
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const float m_new = fmaxf(m_run[nt][e], mx[nt][e]);
-                        const float m_use = m_new == -INFINITY ? 0.f : m_new;
-                        alpha[nt][e] = ex2(m_run[nt][e] - m_use);
-                        m_run[nt][e] = m_new;
-                        mx[nt][e] = m_use;
-                    }
-                }
-                // rows past the end of the context may hold anything (NaN,
-                // Inf): zero this warp's invalid V rows so that 0 * V stays 0
-                if (n_valid < 16 * warp + 16) {
-                    const int first = max(16 * warp, n_valid), last = 16 * warp + 16;
-                    const int lines = (last - first) * C::LINES;
-                    for (int i = lane >> 3; i < lines; i += 4) {
-                        const int tok = first + i / C::LINES, ln = i % C::LINES;
-                        const uint32_t a = sV + (tok / BS) * C::TILE + ln * (BS * 128) +
-                                           (tok % BS) * 128 + (lane & 7) * 16;
-                        sts128(a, 0u, 0u, 0u, 0u);
-                    }
-                    // order these generic-proxy writes before the next TMA
-                    // into the slot
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    __syncwarp();
-                }
-
-                // ---- P^T fragments (B operand, k = token, n = row) ------------
-                // The score accumulator holds S^T[token][row] in the fragment
-                // layout (lane 4r + c: tokens r and r + 8, rows 2c, 2c + 1); a
-                // warp transpose of each 8x8 half gives P^T[row][token] in
-                // the B-operand layout of the PV product.
-                uint32_t pb[NT][2], pl[NT][2];
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    float pr[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) pr[e] = ex2(sacc[nt][e] - mx[nt][e & 1]);
-                    if (!FP8) {
-                        // p = hi + lo, both bf16; the normaliser sums the fp32 p
-                        const uint32_t h0 = pack_bf16x2(pr[0], pr[1]);
-                        const uint32_t h1 = pack_bf16x2(pr[2], pr[3]);
-                        const float2 q0 = unpack_bf16x2(h0), q1 = unpack_bf16x2(h1);
-                        const uint32_t l0 = pack_bf16x2(pr[0] - q0.x, pr[1] - q0.y);
-                        const uint32_t l1 = pack_bf16x2(pr[2] - q1.x, pr[3] - q1.y);
-                        l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + pr[0] + pr[2];
-                        l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + pr[1] + pr[3];
-                        pb[nt][0] = movmatrix_trans(h0);
-                        pb[nt][1] = movmatrix_trans(h1);
-                        pl[nt][0] = movmatrix_trans(l0);
-                        pl[nt][1] = movmatrix_trans(l1);
-                    } else {
-                        // f16 weights; the normaliser sums exactly the rounded values
-                        const uint32_t h0 = pack_f16x2(pr[0], pr[1]);
-                        const uint32_t h1 = pack_f16x2(pr[2], pr[3]);
-                        const float2 q0 = unpack_f16x2(h0), q1 = unpack_f16x2(h1);
-                        l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + q0.x + q1.x;
-                        l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + q0.y + q1.y;
-                        pb[nt][0] = movmatrix_trans(h0);
-                        pb[nt][1] = movmatrix_trans(h1);
-                    }
-                }
-
-                // ---- O^T += V^T . P^T over all D for this warp's tokens ------
-#pragma unroll
-                for (int mt = 0; mt < C::DT; ++mt)
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) o[mt][nt][e] *= alpha[nt][e & 1];
-                if (!FP8) {
-                    const int mi = lane >> 3;
-                    const int tok = 16 * warp + (mi >> 1) * 8 + (lane & 7);
-                    const int row = tok % BS;
-                    const uint32_t rowaddr = sV + (tok / BS) * C::TILE + row * 128;
-#pragma unroll
-                    for (int mt = 0; mt < C::DT; ++mt) {
-                        const int chunk = 2 * mt + (mi & 1);
-                        const uint32_t addr = rowaddr + (chunk >> 3) * (BS * 128) +
-                                              (((chunk & 7) ^ (row & 7)) << 4);
-                        uint32_t a0, a1, a2, a3;
-                        ldsm_x4_t(addr, a0, a1, a2, a3);
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            mma_bf16(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
-                            mma_bf16(o[mt][nt], a0, a1, a2, a3, pl[nt][0], pl[nt][1]);
-                        }
-                    }
-                } else {
-                    // tokens 2c, 2c+1, 2c+8, 2c+9 of this warp; 16 bytes at
-                    // d = 16*gid .. 16*gid + 15 (m-tile mt: bytes 2mt, 2mt+1)
-                    uint32_t wv[4][4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int tok = 16 * warp + 2 * t4 + (q & 1) + (q >> 1) * 8;
-                        const int row = tok % BS;
-                        lds128(sV + (tok / BS) * C::TILE + row * 128 + ((gid ^ (row & 7)) << 4),
-                               wv[q][0], wv[q][1], wv[q][2], wv[q][3]);
-                    }
-#pragma unroll
-                    for (int mt = 0; mt < C::DT; ++mt) {
-                        const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
-                        const uint32_t x = prmt(wv[0][mt >> 1], wv[1][mt >> 1], sel);
-                        const uint32_t y = prmt(wv[2][mt >> 1], wv[3][mt >> 1], sel);
-                        const uint32_t a0 = e4m3x2_to_f16x2(x & 0xffffu);
-                        const uint32_t a1 = e4m3x2_to_f16x2(x >> 16);
-                        const uint32_t a2 = e4m3x2_to_f16x2(y & 0xffffu);
-                        const uint32_t a3 = e4m3x2_to_f16x2(y >> 16);
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
-                            mma_f16(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_empty + 8 * slot);
-        }
-
-        // ---- finish the segment: merge the 4 warps' states -----------------
-        // In a fixed order, so that results do not depend on timing: warps 1
-        // and 3 store their O rows (buffers A and B), warps 0 and 2 add theirs
-        // to them with both weights, and the output is (A + B) / L.
-        // output dim held by accumulator element (mt, e)
-        auto dim_of = [&](int mt, int e) -> int {
-            if (!FP8) return 16 * mt + gid + (e >> 1) * 8;
-            return 16 * gid + 2 * mt + (e >> 1);
-        };
-        // A: warps 0, 1; B: warps 2, 3
-        auto store_rows = [&](int nt) {
-            float *buf = reinterpret_cast<float *>(smem + C::OFF_O + (warp >> 1) * C::OBUF);
-#pragma unroll
-            for (int mt = 0; mt < C::DT; ++mt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    buf[(2 * t4 + (e & 1)) * C::OROW + dim_of(mt, e)] = o[mt][nt][e];
-        };
-        if (warp & 1) store_rows(0);
-        // row sums over this warp's lanes; row max and sum of every warp
-        // through shared memory; all consumers agree on leaving after a timeout
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                float v = l_run[nt][e];
-#pragma unroll
-                for (int off = 4; off < 32; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-                if (gid == 0) {
-                    red[warp * C::NP + nt * 8 + 2 * t4 + e] = m_run[nt][e];
-                    lsum[warp * C::NP + nt * 8 + 2 * t4 + e] = v;
-                }
-            }
-        if (named_bar_sync_or(kBarConsumers, kConsumers, abort)) return;
-        // weights of this warp's and its partner's (warp + 1) O in the merged row
-        float wsc[NT][2], psc[NT][2];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int r = nt * 8 + 2 * t4 + e;
-                float M = -INFINITY;
-#pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[w * C::NP + r]);
-                const float Mu = M == -INFINITY ? 0.f : M;
-                wsc[nt][e] = ex2(m_run[nt][e] - Mu);
-                psc[nt][e] = ex2(red[((warp + 1) & 3) * C::NP + r] - Mu);
-                if (warp == 0 && gid == 0) {
-                    float L = 0.f;
-#pragma unroll
-                    for (int w = 0; w < kConsumerWarps; ++w)
-                        L += lsum[w * C::NP + r] * ex2(red[w * C::NP + r] - Mu);
-                    rowinv[r] = L > 0.f ? vsc / L : 0.f;
-                    rowlse[r] = L > 0.f ? M + log2f(L) : -INFINITY;
-                }
-            }
-
         // output row of query row r: query token r / g, head h*g + r % g
         auto orow = [&](int r) -> long long {
             return ((long long)s * p.q_len + r / g) * p.num_q_heads + (long long)h * g + r % g;
@@ -1113,31 +805,9 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         // partial results: slot 2c for the CTA's first segment, 2c+1 for its last
         const long long pslot = 2 * cta + (useg == u0 ? 0 : 1);
         constexpr int CPR = D / 8;   // 8-float chunks per row
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            if (nt > 0) {
-                named_bar_sync(kBarConsumers, kConsumers);   // A and B read
-                if (warp & 1) store_rows(nt);
-                named_bar_sync(kBarConsumers, kConsumers);
-            }
-            // warps 0 and 2: buffer = own O * weight + partner's O * its weight
-            if (!(warp & 1)) {
-                float *buf = reinterpret_cast<float *>(smem + C::OFF_O + (warp >> 1) * C::OBUF);
-                float part[C::DT][4];
-#pragma unroll
-                for (int mt = 0; mt < C::DT; ++mt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        part[mt][e] = buf[(2 * t4 + (e & 1)) * C::OROW + dim_of(mt, e)];
-#pragma unroll
-                for (int mt = 0; mt < C::DT; ++mt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        buf[(2 * t4 + (e & 1)) * C::OROW + dim_of(mt, e)] =
-                            o[mt][nt][e] * wsc[nt][e & 1] + part[mt][e] * psc[nt][e & 1];
-            }
-            named_bar_sync(kBarConsumers, kConsumers);
-            // (A + B) / L, 8 consecutive dims per step
+        // (A + B) / L for the rows of round nt (rows 8*nt .. 8*nt + 7), 8
+        // consecutive dims per step: the output, or this CTA's partial result
+        auto finalize_rows = [&](int nt) {
             for (int c = tid; c < 8 * CPR; c += kConsumers) {
                 const int rl = c / CPR, d0 = (c % CPR) * 8, r = nt * 8 + rl;
                 if (r >= R) continue;
@@ -1174,6 +844,549 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     if (d0 == 0) p.lse_part[pslot * R + r] = rowlse[r];
                 }
             }
+        };
+
+        if constexpr (CC == 0) {
+            // visible token range [lo, hi) of the two query rows this lane holds
+            // per n-tile (rows 8*nt + 2*t4 + {0, 1}; row = query token * g + head)
+            int vis_lo[NT][2], vis_hi[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int row = nt * 8 + 2 * t4 + e;
+                    const int hi = ctx - p.q_len + 1 + row / g;
+                    vis_hi[nt][e] = row < R ? hi : 0;
+                    vis_lo[nt][e] = (row < R && p.window > 0) ? max(0, hi - p.window) : 0;
+                }
+
+            // query fragments (B operand, Q^T[d][row]) from the slot
+            uint32_t qf[C::KSTEPS][NT][2];
+            {
+                const uint32_t qb = sQ + qs * C::QSLOT;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int head = nt * 8 + gid;      // query row held as B column
+                    const bool live = head < R;
+                    const uint32_t qr = qb + (live ? head : 0) * D * 2;
+#pragma unroll
+                    for (int k = 0; k < C::KSTEPS; ++k) {
+                        uint32_t b0, b1;
+                        if (!FP8) {   // k index 2t, 2t+1 | 2t+8, 2t+9  <->  same d
+                            b0 = lds32(qr + (16 * k + 2 * t4) * 2);
+                            b1 = lds32(qr + (16 * k + 8 + 2 * t4) * 2);
+                        } else {      // k index permuted to d = 16k + 4t + {0,1 | 2,3}
+                            b0 = bf16x2_to_f16x2(lds32(qr + (16 * k + 4 * t4) * 2));
+                            b1 = bf16x2_to_f16x2(lds32(qr + (16 * k + 4 * t4 + 2) * 2));
+                        }
+                        qf[k][nt][0] = live ? b0 : 0u;
+                        qf[k][nt][1] = live ? b1 : 0u;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(seg_empty + 8 * qs);   // the slot may be refilled
+            ++sit;
+
+
+            // This warp's online-softmax state over its own 16 tokens of every
+            // stage: running max and (lane-partial) sum per query row, and
+            // O^T[d][row] for all D dims.  The 4 warps' states are merged once,
+            // at the end of the segment.
+            float m_run[NT][2], l_run[NT][2];
+            float o[C::DT][NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                m_run[nt][0] = m_run[nt][1] = -INFINITY;
+                l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+                for (int mt = 0; mt < C::DT; ++mt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
+            }
+
+            bool abort = false;
+            for (int jj = j0; jj < j1; jj += C::BPS) {
+                const int nb = min(C::BPS, j1 - jj);
+                // tokens of the stage that were loaded (the stage may end with the
+                // segment or with the context)
+                const int n_valid = min(ctx - jj * BS, nb * BS);
+                const uint32_t slot = it % NSTAGES;
+                const bool ok = mbar_wait_bounded(bar_full + 8 * slot, (it / NSTAGES) & 1);
+                ++it;
+                if (!ok) {
+                    raise_flag(p.flags, kFlagTimeout);
+                    abort = true;
+                    break;
+                }
+                const uint32_t sK = sbase + slot * C::STAGE, sV = sK + C::STAGE_KV;
+
+                if (16 * warp < n_valid) {
+                    // ---- S^T = K . Q^T for this warp's 16 tokens (two MMA chains)
+                    float sacc[NT][4], sac2[NT][4];
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) sacc[nt][e] = sac2[nt][e] = 0.f;
+                    if (!FP8) {
+                        const int mi = lane >> 3;
+                        const int tok = 16 * warp + (mi & 1) * 8 + (lane & 7);
+                        const int row = tok % BS;
+                        const uint32_t rowaddr = sK + (tok / BS) * C::TILE + row * 128;
+#pragma unroll
+                        for (int k = 0; k < C::KSTEPS; ++k) {
+                            const int chunk = 2 * k + (mi >> 1);
+                            const uint32_t addr = rowaddr + (chunk >> 3) * (BS * 128) +
+                                                  (((chunk & 7) ^ (row & 7)) << 4);
+                            uint32_t a0, a1, a2, a3;
+                            ldsm_x4(addr, a0, a1, a2, a3);
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt) {
+                                if (k & 1) mma_bf16(sac2[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
+                                else       mma_bf16(sacc[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
+                            }
+                        }
+                    } else {
+                        const int tok0 = 16 * warp + gid, tok1 = tok0 + 8;
+                        const int r0 = tok0 % BS, r1 = tok1 % BS;
+                        const uint32_t base0 = sK + (tok0 / BS) * C::TILE + r0 * 128 + 4 * t4;
+                        const uint32_t base1 = sK + (tok1 / BS) * C::TILE + r1 * 128 + 4 * t4;
+#pragma unroll
+                        for (int k = 0; k < C::KSTEPS; ++k) {
+                            const uint32_t w0 = lds32(base0 + ((k ^ (r0 & 7)) << 4));
+                            const uint32_t w1 = lds32(base1 + ((k ^ (r1 & 7)) << 4));
+                            const uint32_t a0 = e4m3x2_to_f16x2(w0 & 0xffffu);
+                            const uint32_t a2 = e4m3x2_to_f16x2(w0 >> 16);
+                            const uint32_t a1 = e4m3x2_to_f16x2(w1 & 0xffffu);
+                            const uint32_t a3 = e4m3x2_to_f16x2(w1 >> 16);
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt) {
+                                if (k & 1) mma_f16(sac2[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
+                                else       mma_f16(sacc[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
+                            }
+                        }
+                    }
+
+                    // ---- mask, this warp's max per row, weights p ----------------
+                    float mx[NT][2], alpha[NT][2];
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            // stage token (only the first n_valid were loaded) and
+                            // its absolute position; the row's visible range
+                            // excludes padding rows and positions past ctx
+                            const int tok = 16 * warp + gid + (e >> 1) * 8;
+                            const int pos = jj * BS + tok;
+                            const float v = sacc[nt][e] + sac2[nt][e];
+                            sacc[nt][e] = (tok < n_valid && pos >= vis_lo[nt][e & 1] &&
+                                           pos < vis_hi[nt][e & 1])
+                                              ? v * sl2 : -INFINITY;
+                        }
+                        mx[nt][0] = fmaxf(sacc[nt][0], sacc[nt][2]);
+                        mx[nt][1] = fmaxf(sacc[nt][1], sacc[nt][3]);
+#pragma unroll
+                        for (int off = 4; off < 32; off <<= 1) {
+                            mx[nt][0] = fmaxf(mx[nt][0], __shfl_xor_sync(0xffffffffu, mx[nt][0], off));
+                            mx[nt][1] = fmaxf(mx[nt][1], __shfl_xor_sync(0xffffffffu, mx[nt][1], off));
+                        }
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const float m_new = fmaxf(m_run[nt][e], mx[nt][e]);
+                            const float m_use = m_new == -INFINITY ? 0.f : m_new;
+                            alpha[nt][e] = ex2(m_run[nt][e] - m_use);
+                            m_run[nt][e] = m_new;
+                            mx[nt][e] = m_use;
+                        }
+                    }
+                    // rows past the end of the context may hold anything (NaN,
+                    // Inf): zero this warp's invalid V rows so that 0 * V stays 0
+                    if (n_valid < 16 * warp + 16) {
+                        const int first = max(16 * warp, n_valid), last = 16 * warp + 16;
+                        const int lines = (last - first) * C::LINES;
+                        for (int i = lane >> 3; i < lines; i += 4) {
+                            const int tok = first + i / C::LINES, ln = i % C::LINES;
+                            const uint32_t a = sV + (tok / BS) * C::TILE + ln * (BS * 128) +
+                                               (tok % BS) * 128 + (lane & 7) * 16;
+                            sts128(a, 0u, 0u, 0u, 0u);
+                        }
+                        // order these generic-proxy writes before the next TMA
+                        // into the slot
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        __syncwarp();
+                    }
+
+                    // ---- P^T fragments (B operand, k = token, n = row) ------------
+                    // The score accumulator holds S^T[token][row] in the fragment
+                    // layout (lane 4r + c: tokens r and r + 8, rows 2c, 2c + 1); a
+                    // warp transpose of each 8x8 half gives P^T[row][token] in
+                    // the B-operand layout of the PV product.
+                    uint32_t pb[NT][2], pl[NT][2];
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        float pr[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) pr[e] = ex2(sacc[nt][e] - mx[nt][e & 1]);
+                        if (!FP8) {
+                            // p = hi + lo, both bf16; the normaliser sums the fp32 p
+                            const uint32_t h0 = pack_bf16x2(pr[0], pr[1]);
+                            const uint32_t h1 = pack_bf16x2(pr[2], pr[3]);
+                            const float2 q0 = unpack_bf16x2(h0), q1 = unpack_bf16x2(h1);
+                            const uint32_t l0 = pack_bf16x2(pr[0] - q0.x, pr[1] - q0.y);
+                            const uint32_t l1 = pack_bf16x2(pr[2] - q1.x, pr[3] - q1.y);
+                            l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + pr[0] + pr[2];
+                            l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + pr[1] + pr[3];
+                            pb[nt][0] = movmatrix_trans(h0);
+                            pb[nt][1] = movmatrix_trans(h1);
+                            pl[nt][0] = movmatrix_trans(l0);
+                            pl[nt][1] = movmatrix_trans(l1);
+                        } else {
+                            // f16 weights; the normaliser sums exactly the rounded values
+                            const uint32_t h0 = pack_f16x2(pr[0], pr[1]);
+                            const uint32_t h1 = pack_f16x2(pr[2], pr[3]);
+                            const float2 q0 = unpack_f16x2(h0), q1 = unpack_f16x2(h1);
+                            l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + q0.x + q1.x;
+                            l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + q0.y + q1.y;
+                            pb[nt][0] = movmatrix_trans(h0);
+                            pb[nt][1] = movmatrix_trans(h1);
+                        }
+                    }
+
+                    // ---- O^T += V^T . P^T over all D for this warp's tokens ------
+#pragma unroll
+                    for (int mt = 0; mt < C::DT; ++mt)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) o[mt][nt][e] *= alpha[nt][e & 1];
+                    if (!FP8) {
+                        const int mi = lane >> 3;
+                        const int tok = 16 * warp + (mi >> 1) * 8 + (lane & 7);
+                        const int row = tok % BS;
+                        const uint32_t rowaddr = sV + (tok / BS) * C::TILE + row * 128;
+#pragma unroll
+                        for (int mt = 0; mt < C::DT; ++mt) {
+                            const int chunk = 2 * mt + (mi & 1);
+                            const uint32_t addr = rowaddr + (chunk >> 3) * (BS * 128) +
+                                                  (((chunk & 7) ^ (row & 7)) << 4);
+                            uint32_t a0, a1, a2, a3;
+                            ldsm_x4_t(addr, a0, a1, a2, a3);
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt) {
+                                mma_bf16(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+                                mma_bf16(o[mt][nt], a0, a1, a2, a3, pl[nt][0], pl[nt][1]);
+                            }
+                        }
+                    } else {
+                        // tokens 2c, 2c+1, 2c+8, 2c+9 of this warp; 16 bytes at
+                        // d = 16*gid .. 16*gid + 15 (m-tile mt: bytes 2mt, 2mt+1)
+                        uint32_t wv[4][4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int tok = 16 * warp + 2 * t4 + (q & 1) + (q >> 1) * 8;
+                            const int row = tok % BS;
+                            lds128(sV + (tok / BS) * C::TILE + row * 128 + ((gid ^ (row & 7)) << 4),
+                                   wv[q][0], wv[q][1], wv[q][2], wv[q][3]);
+                        }
+#pragma unroll
+                        for (int mt = 0; mt < C::DT; ++mt) {
+                            const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+                            const uint32_t x = prmt(wv[0][mt >> 1], wv[1][mt >> 1], sel);
+                            const uint32_t y = prmt(wv[2][mt >> 1], wv[3][mt >> 1], sel);
+                            const uint32_t a0 = e4m3x2_to_f16x2(x & 0xffffu);
+                            const uint32_t a1 = e4m3x2_to_f16x2(x >> 16);
+                            const uint32_t a2 = e4m3x2_to_f16x2(y & 0xffffu);
+                            const uint32_t a3 = e4m3x2_to_f16x2(y >> 16);
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt)
+                                mma_f16(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_empty + 8 * slot);
+            }
+
+            // ---- finish the segment: merge the 4 warps' states -----------------
+            // In a fixed order, so that results do not depend on timing: warps 1
+            // and 3 store their O rows (buffers A and B), warps 0 and 2 add theirs
+            // to them with both weights, and the output is (A + B) / L.
+            // output dim held by accumulator element (mt, e)
+            auto dim_of = [&](int mt, int e) -> int {
+                if (!FP8) return 16 * mt + gid + (e >> 1) * 8;
+                return 16 * gid + 2 * mt + (e >> 1);
+            };
+            // A: warps 0, 1; B: warps 2, 3
+            auto store_rows = [&](int nt) {
+                float *buf = reinterpret_cast<float *>(smem + C::OFF_O + (warp >> 1) * C::OBUF);
+#pragma unroll
+                for (int mt = 0; mt < C::DT; ++mt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        buf[(2 * t4 + (e & 1)) * C::OROW + dim_of(mt, e)] = o[mt][nt][e];
+            };
+            if (warp & 1) store_rows(0);
+            // row sums over this warp's lanes; row max and sum of every warp
+            // through shared memory; all consumers agree on leaving after a timeout
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    float v = l_run[nt][e];
+#pragma unroll
+                    for (int off = 4; off < 32; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                    if (gid == 0) {
+                        red[warp * C::NP + nt * 8 + 2 * t4 + e] = m_run[nt][e];
+                        lsum[warp * C::NP + nt * 8 + 2 * t4 + e] = v;
+                    }
+                }
+            if (named_bar_sync_or(kBarConsumers, kConsumers, abort)) return;
+            // weights of this warp's and its partner's (warp + 1) O in the merged row
+            float wsc[NT][2], psc[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int r = nt * 8 + 2 * t4 + e;
+                    float M = -INFINITY;
+#pragma unroll
+                    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[w * C::NP + r]);
+                    const float Mu = M == -INFINITY ? 0.f : M;
+                    wsc[nt][e] = ex2(m_run[nt][e] - Mu);
+                    psc[nt][e] = ex2(red[((warp + 1) & 3) * C::NP + r] - Mu);
+                    if (warp == 0 && gid == 0) {
+                        float L = 0.f;
+#pragma unroll
+                        for (int w = 0; w < kConsumerWarps; ++w)
+                            L += lsum[w * C::NP + r] * ex2(red[w * C::NP + r] - Mu);
+                        rowinv[r] = L > 0.f ? vsc / L : 0.f;
+                        rowlse[r] = L > 0.f ? M + log2f(L) : -INFINITY;
+                    }
+                }
+
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                if (nt > 0) {
+                    named_bar_sync(kBarConsumers, kConsumers);   // A and B read
+                    if (warp & 1) store_rows(nt);
+                    named_bar_sync(kBarConsumers, kConsumers);
+                }
+                // warps 0 and 2: buffer = own O * weight + partner's O * its weight
+                if (!(warp & 1)) {
+                    float *buf = reinterpret_cast<float *>(smem + C::OFF_O + (warp >> 1) * C::OBUF);
+                    float part[C::DT][4];
+#pragma unroll
+                    for (int mt = 0; mt < C::DT; ++mt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            part[mt][e] = buf[(2 * t4 + (e & 1)) * C::OROW + dim_of(mt, e)];
+#pragma unroll
+                    for (int mt = 0; mt < C::DT; ++mt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            buf[(2 * t4 + (e & 1)) * C::OROW + dim_of(mt, e)] =
+                                o[mt][nt][e] * wsc[nt][e & 1] + part[mt][e] * psc[nt][e & 1];
+                }
+                named_bar_sync(kBarConsumers, kConsumers);
+                finalize_rows(nt);
+            }
+        } else {
+            // ---- CUDA-core variant: FMA dot products, warp-shuffle sums --------
+            // Lane l owns dims 4l .. 4l+3 of every query row (head_dim 128).
+            // For a group of TG tokens each lane forms the partial dot products
+            // of its 4 dims for all TG x CC (token, row) pairs; a butterfly of
+            // shuffles leaves lane l the full score of pair l (token l / CC,
+            // row l % CC).  P goes through this warp's shared-memory area to
+            // every lane, which accumulates O for its 4 dims of every row.
+            constexpr int RP = CC, TG = 32 / RP, NGR = 16 / TG;
+            const int my_r = lane % RP;            // the row of the scores this lane holds
+            int vlo, vhi;
+            {
+                const int hi = ctx - p.q_len + 1 + my_r / g;
+                vhi = my_r < R ? hi : 0;
+                vlo = (my_r < R && p.window > 0) ? max(0, hi - p.window) : 0;
+            }
+            // dims 4l .. 4l+3 of bf16 row `tok` of a K or V stage, as fp32
+            auto load4 = [&](uint32_t tile0, int tok, float (&v)[4]) {
+                const int row = tok % BS;
+                const uint32_t a = tile0 + (tok / BS) * C::TILE + (lane >> 4) * (BS * 128) +
+                                   row * 128 + ((((lane & 15) >> 1) ^ (row & 7)) << 4) +
+                                   8 * (lane & 1);
+                const long long w = lds64(a);
+                const uint32_t x = (uint32_t)w, y = (uint32_t)(w >> 32);
+                v[0] = __uint_as_float(x << 16);
+                v[1] = __uint_as_float(x & 0xFFFF0000u);
+                v[2] = __uint_as_float(y << 16);
+                v[3] = __uint_as_float(y & 0xFFFF0000u);
+            };
+            float qv[RP][4];
+            {
+                const uint32_t qb = sQ + qs * C::QSLOT;
+#pragma unroll
+                for (int r = 0; r < RP; ++r) {
+                    const long long w = lds64(qb + (min(r, R - 1) * D + 4 * lane) * 2);
+                    const uint32_t x = (uint32_t)w, y = (uint32_t)(w >> 32);
+                    const bool live = r < R;
+                    qv[r][0] = live ? __uint_as_float(x << 16) : 0.f;
+                    qv[r][1] = live ? __uint_as_float(x & 0xFFFF0000u) : 0.f;
+                    qv[r][2] = live ? __uint_as_float(y << 16) : 0.f;
+                    qv[r][3] = live ? __uint_as_float(y & 0xFFFF0000u) : 0.f;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(seg_empty + 8 * qs);   // the slot may be refilled
+            ++sit;
+
+            float o4[RP][4];
+#pragma unroll
+            for (int r = 0; r < RP; ++r)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) o4[r][j] = 0.f;
+            float m_my = -INFINITY, l_my = 0.f;   // this lane's row: running max, its share of the sum
+            float *pw = reinterpret_cast<float *>(smem + C::OFF_PW) + warp * C::PWF;
+            bool abort = false;
+            for (int jj = j0; jj < j1; jj += C::BPS) {
+                const int nb = min(C::BPS, j1 - jj);
+                const int n_valid = min(ctx - jj * BS, nb * BS);
+                const uint32_t slot = it % NSTAGES;
+                const bool ok = mbar_wait_bounded(bar_full + 8 * slot, (it / NSTAGES) & 1);
+                ++it;
+                if (!ok) {
+                    raise_flag(p.flags, kFlagTimeout);
+                    abort = true;
+                    break;
+                }
+                const uint32_t sK = sbase + slot * C::STAGE, sV = sK + C::STAGE_KV;
+                const int nv = n_valid - 16 * warp;   // loaded tokens of this warp (uniform)
+                if (nv > 0) {
+                    float sc[NGR];
+#pragma unroll
+                    for (int gi = 0; gi < NGR; ++gi) {
+                        float acc[32];
+#pragma unroll
+                        for (int tt = 0; tt < TG; ++tt) {
+                            const int tk = gi * TG + tt;
+                            float k4[4] = {0.f, 0.f, 0.f, 0.f};
+                            if (tk < nv) load4(sK, 16 * warp + tk, k4);
+#pragma unroll
+                            for (int r = 0; r < RP; ++r)
+                                acc[tt * RP + r] = qv[r][0] * k4[0] + qv[r][1] * k4[1] +
+                                                   qv[r][2] * k4[2] + qv[r][3] * k4[3];
+                        }
+                        // reduce-scatter over the 32 lanes: lane l keeps entry l
+#pragma unroll
+                        for (int off = 16, len = 32; off >= 1; off >>= 1, len >>= 1) {
+                            const bool up = (lane & off) != 0;
+#pragma unroll
+                            for (int i = 0; i < len / 2; ++i) {
+                                const float send = up ? acc[i] : acc[i + len / 2];
+                                const float keep = up ? acc[i + len / 2] : acc[i];
+                                acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                            }
+                        }
+                        const int tk = gi * TG + lane / RP;
+                        const int pos = jj * BS + 16 * warp + tk;
+                        sc[gi] = (tk < nv && pos >= vlo && pos < vhi) ? acc[0] * sl2 : -INFINITY;
+                    }
+                    // this stage's max of the lane's row (lanes with the same row)
+                    float mx = sc[0];
+#pragma unroll
+                    for (int gi = 1; gi < NGR; ++gi) mx = fmaxf(mx, sc[gi]);
+#pragma unroll
+                    for (int off = RP; off < 32; off <<= 1)
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                    const float m_new = fmaxf(m_my, mx);
+                    const float m_use = m_new == -INFINITY ? 0.f : m_new;
+                    const float al = ex2(m_my - m_use);
+                    m_my = m_new;
+                    float ps = 0.f;
+#pragma unroll
+                    for (int gi = 0; gi < NGR; ++gi) {
+                        const float pv = ex2(sc[gi] - m_use);
+                        ps += pv;
+                        pw[(gi * TG + lane / RP) * RP + my_r] = pv;
+                    }
+                    l_my = l_my * al + ps;
+                    if (lane < RP) pw[16 * RP + lane] = al;
+                    __syncwarp();
+                    // rescale O and add this warp's tokens
+#pragma unroll
+                    for (int r = 0; r < RP; ++r) {
+                        const float a = pw[16 * RP + r];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) o4[r][j] *= a;
+                    }
+                    for (int tk = 0; tk < min(nv, 16); ++tk) {
+                        float v4[4];
+                        load4(sV, 16 * warp + tk, v4);
+#pragma unroll
+                        for (int r4 = 0; r4 < RP / 4; ++r4) {
+                            const float4 pr = reinterpret_cast<const float4 *>(pw + tk * RP)[r4];
+                            const float pp[4] = {pr.x, pr.y, pr.z, pr.w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) o4[4 * r4 + i][j] += pp[i] * v4[j];
+                        }
+                    }
+                    __syncwarp();   // pw is rewritten by the next stage
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_empty + 8 * slot);
+            }
+
+            // ---- merge the 4 warps' states (same fixed order as above) --------
+            float *buf = reinterpret_cast<float *>(smem + C::OFF_O + (warp >> 1) * C::OBUF);
+            if (warp & 1) {
+#pragma unroll
+                for (int r = 0; r < RP; ++r)
+                    *reinterpret_cast<float4 *>(buf + r * C::OROW + 4 * lane) =
+                        make_float4(o4[r][0], o4[r][1], o4[r][2], o4[r][3]);
+            }
+            float lr = l_my;
+#pragma unroll
+            for (int off = RP; off < 32; off <<= 1) lr += __shfl_xor_sync(0xffffffffu, lr, off);
+            if (lane < C::NP) {       // lane r < RP holds row r
+                red[warp * C::NP + lane] = lane < RP ? m_my : -INFINITY;
+                lsum[warp * C::NP + lane] = lane < RP ? lr : 0.f;
+            }
+            if (named_bar_sync_or(kBarConsumers, kConsumers, abort)) return;
+            float wsc[RP], psc[RP];
+#pragma unroll
+            for (int r = 0; r < RP; ++r) {
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[w * C::NP + r]);
+                const float Mu = M == -INFINITY ? 0.f : M;
+                wsc[r] = ex2(red[warp * C::NP + r] - Mu);
+                psc[r] = ex2(red[((warp + 1) & 3) * C::NP + r] - Mu);
+            }
+            if (warp == 0 && lane < C::NP) {
+                const int r = lane;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[w * C::NP + r]);
+                const float Mu = M == -INFINITY ? 0.f : M;
+                float L = 0.f;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w)
+                    L += lsum[w * C::NP + r] * ex2(red[w * C::NP + r] - Mu);
+                rowinv[r] = L > 0.f ? vsc / L : 0.f;
+                rowlse[r] = L > 0.f ? M + log2f(L) : -INFINITY;
+            }
+            if (!(warp & 1)) {
+#pragma unroll
+                for (int r = 0; r < RP; ++r) {
+                    float4 *b4 = reinterpret_cast<float4 *>(buf + r * C::OROW + 4 * lane);
+                    const float4 q4 = *b4;
+                    *b4 = make_float4(o4[r][0] * wsc[r] + q4.x * psc[r],
+                                      o4[r][1] * wsc[r] + q4.y * psc[r],
+                                      o4[r][2] * wsc[r] + q4.z * psc[r],
+                                      o4[r][3] * wsc[r] + q4.w * psc[r]);
+                }
+            }
+            named_bar_sync(kBarConsumers, kConsumers);
+            finalize_rows(0);
         }
         if (!whole) {
             // every consumer's partial stores precede the barrier; the arrival

@@ -24,11 +24,12 @@ struct Stages {
     static constexpr int value = FP8 ? 6 : 3;
 };
 
-template <int D, int BS, int NT, bool FP8>
+// CC = 0: tensor-core consumers; CC = 4 / 8: the CUDA-core comparison variant
+template <int D, int BS, int NT, bool FP8, int CC = 0>
 cudaError_t launch_decode(const DecodeLaunchArgs &a);
 
 // Resident CTAs per SM for this variant (0 if it cannot launch).
-template <int D, int BS, int NT, bool FP8>
+template <int D, int BS, int NT, bool FP8, int CC = 0>
 int decode_ctas_per_sm();
 
 #define PGD_DECLARE_FAMILY(D, FP8)                                                    \
@@ -48,6 +49,17 @@ int decode_ctas_per_sm();
 PGD_DECLARE_FAMILY(128, false)
 PGD_DECLARE_FAMILY(256, false)
 PGD_DECLARE_FAMILY(128, true)
+
+#define PGD_DECLARE_CUDA_CORE(CC)                                                         \
+    extern template cudaError_t launch_decode<128, 16, 1, false, CC>(const DecodeLaunchArgs &); \
+    extern template cudaError_t launch_decode<128, 32, 1, false, CC>(const DecodeLaunchArgs &); \
+    extern template cudaError_t launch_decode<128, 64, 1, false, CC>(const DecodeLaunchArgs &); \
+    extern template int decode_ctas_per_sm<128, 16, 1, false, CC>();                           \
+    extern template int decode_ctas_per_sm<128, 32, 1, false, CC>();                           \
+    extern template int decode_ctas_per_sm<128, 64, 1, false, CC>();
+
+PGD_DECLARE_CUDA_CORE(4)
+PGD_DECLARE_CUDA_CORE(8)
 
 // kv_append and the standalone LSE merge (pgd_aux.cu)
 cudaError_t launch_kv_append(const void *k_new, const void *v_new, const int64_t *slots,

@@ -167,3 +167,12 @@ def test_partial_decode_needs_lse(lib):
     assert lib.pgd_paged_decode_partial(*args, MIS, A, None, 0, 0, None) == INVALID
     args[6] = 0   # empty batch
     assert lib.pgd_paged_decode_partial(*args, None, None, None, 0, 0, None) == OK
+
+
+def test_decode_math_setting_is_host_only(lib):
+    lib.pgd_set_decode_math.argtypes = [ctypes.c_int]
+    lib.pgd_get_decode_math.restype = ctypes.c_int
+    assert lib.pgd_get_decode_math() == 0
+    assert lib.pgd_set_decode_math(1) == OK and lib.pgd_get_decode_math() == 1
+    assert lib.pgd_set_decode_math(7) == INVALID and lib.pgd_get_decode_math() == 1
+    assert lib.pgd_set_decode_math(0) == OK and lib.pgd_get_decode_math() == 0
