@@ -87,6 +87,9 @@ constexpr int kThreads = kConsumers + 64;   // + producer warp + appender warp
 constexpr int kAppSlots = 4;                // appender -> producer handoff ring
 constexpr int kStageTokens = 16 * kConsumerWarps;
 constexpr float kLn2 = 0.6931471805599453f;
+// log2 of the largest softmax weight a consumer lets accumulate before it
+// moves a row's reference max (lazy rescaling)
+constexpr float kLazyRescale = 8.f;
 constexpr uint32_t kBarConsumers = 1;
 
 // Segment descriptor written by the producer, read by the consumers.
@@ -990,15 +993,30 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                             mx[nt][0] = fmaxf(mx[nt][0], __shfl_xor_sync(0xffffffffu, mx[nt][0], off));
                             mx[nt][1] = fmaxf(mx[nt][1], __shfl_xor_sync(0xffffffffu, mx[nt][1], off));
                         }
+                    }
+                    // Lazy rescaling: a row keeps its reference max m_run (the
+                    // exponent offset of every weight it has summed) until a
+                    // score exceeds it by more than 2^8, so weights stay below
+                    // 256 and the accumulator is rescaled only in the stages
+                    // where some row of the warp moves.
+                    bool moved = false;
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e)
+                            moved |= mx[nt][e] > m_run[nt][e] + kLazyRescale;
+                    const bool any_moved = __any_sync(0xffffffffu, moved);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                         for (int e = 0; e < 2; ++e) {
-                            const float m_new = fmaxf(m_run[nt][e], mx[nt][e]);
-                            const float m_use = m_new == -INFINITY ? 0.f : m_new;
-                            alpha[nt][e] = ex2(m_run[nt][e] - m_use);
-                            m_run[nt][e] = m_new;
-                            mx[nt][e] = m_use;
+                            alpha[nt][e] = 1.f;
+                            if (any_moved && mx[nt][e] > m_run[nt][e] + kLazyRescale) {
+                                alpha[nt][e] = ex2(m_run[nt][e] - mx[nt][e]);
+                                m_run[nt][e] = mx[nt][e];
+                            }
+                            mx[nt][e] = m_run[nt][e] == -INFINITY ? 0.f : m_run[nt][e];
                         }
-                    }
                     // rows past the end of the context may hold anything (NaN,
                     // Inf): zero this warp's invalid V rows so that 0 * V stays 0
                     if (n_valid < 16 * warp + 16) {
@@ -1053,12 +1071,14 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     }
 
                     // ---- O^T += V^T . P^T over all D for this warp's tokens ------
+                    if (any_moved) {
 #pragma unroll
-                    for (int mt = 0; mt < C::DT; ++mt)
+                        for (int mt = 0; mt < C::DT; ++mt)
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
+                            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) o[mt][nt][e] *= alpha[nt][e & 1];
+                                for (int e = 0; e < 4; ++e) o[mt][nt][e] *= alpha[nt][e & 1];
+                    }
                     if (!FP8) {
                         const int mi = lane >> 3;
                         const int tok = 16 * warp + (mi >> 1) * 8 + (lane & 7);
