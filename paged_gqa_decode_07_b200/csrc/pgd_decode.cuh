@@ -116,7 +116,12 @@ struct DecodeCfg {
     static constexpr int NP = 8 * NT;                    // padded query rows per unit
     static constexpr int DT = D / 16;                    // PV m-tiles (each warp: all of D)
     static constexpr int KSTEPS = D / 16;                // QK k-steps
-    static constexpr int QSLOT = NP * D * 2;             // query rows of one unit
+    // head_dim 256 with tensor cores: the query rows stay in shared memory
+    // for the whole segment (row stride padded by 16 bytes so that an
+    // ldmatrix of 8 rows hits 8 bank groups) instead of in registers
+    static constexpr bool QSMEM = D == 256 && !FP8 && CC == 0;
+    static constexpr int QROW = QSMEM ? D * 2 + 16 : D * 2;
+    static constexpr int QSLOT = NP * QROW;              // query rows of one unit
     // descriptor ring depth (one slot for 16 query rows at head_dim 128, so
     // that two CTAs still fit on an SM)
     static constexpr int NSEG = CC ? 2 : (D == 128 ? (QSLOT >= 4096 ? 1 : 3) : 2);
@@ -687,11 +692,21 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     const uint32_t bar = seg_full + 8 * slot;
                     mbar_arrive_expect_tx(bar, qtok * p.q_len);
                     // query rows: q_len runs of g contiguous heads, row = i*g + head
-                    for (int i = 0; i < p.q_len; ++i)
-                        bulk_copy_g2s(sQ + slot * C::QSLOT + i * qtok,
-                                      p.q + (((long long)cur.s * p.q_len + i) * p.num_q_heads +
-                                             (long long)cur.h * g) * D,
-                                      qtok, bar);
+                    if (!C::QSMEM)
+                        for (int i = 0; i < p.q_len; ++i)
+                            bulk_copy_g2s(sQ + slot * C::QSLOT + i * qtok,
+                                          p.q + (((long long)cur.s * p.q_len + i) * p.num_q_heads +
+                                                 (long long)cur.h * g) * D,
+                                          qtok, bar);
+                }
+                if (C::QSMEM) {
+                    // one copy per row into the padded slot (after the expect-tx)
+                    __syncwarp();
+                    for (int r = lane; r < g * p.q_len; r += 32)
+                        bulk_copy_g2s(sQ + slot * C::QSLOT + r * C::QROW,
+                                      p.q + (((long long)cur.s * p.q_len + r / g) * p.num_q_heads +
+                                             (long long)cur.h * g + r % g) * D,
+                                      D * 2, seg_full + 8 * slot);
                 }
                 ++sit;
             }
@@ -863,10 +878,12 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     vis_lo[nt][e] = (row < R && p.window > 0) ? max(0, hi - p.window) : 0;
                 }
 
-            // query fragments (B operand, Q^T[d][row]) from the slot
-            uint32_t qf[C::KSTEPS][NT][2];
-            {
-                const uint32_t qb = sQ + qs * C::QSLOT;
+            // query fragments (B operand, Q^T[d][row]) from the slot: into
+            // registers now, or (head_dim 256) by ldmatrix at every k-step
+            const uint32_t qbase = sQ + qs * C::QSLOT;
+            uint32_t qf[C::QSMEM ? 1 : C::KSTEPS][NT][2];
+            if constexpr (!C::QSMEM) {
+                const uint32_t qb = qbase;
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const int head = nt * 8 + gid;      // query row held as B column
@@ -887,10 +904,11 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     }
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(seg_empty + 8 * qs);   // the slot may be refilled
+            if (!C::QSMEM) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(seg_empty + 8 * qs);   // the slot may be refilled
+            }
             ++sit;
-
 
             // This warp's online-softmax state over its own 16 tokens of every
             // stage: running max and (lane-partial) sum per query row, and
@@ -936,6 +954,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                         const int tok = 16 * warp + (mi & 1) * 8 + (lane & 7);
                         const int row = tok % BS;
                         const uint32_t rowaddr = sK + (tok / BS) * C::TILE + row * 128;
+                        uint32_t qb4[NT][4];   // shared-memory query fragments of k, k + 1
 #pragma unroll
                         for (int k = 0; k < C::KSTEPS; ++k) {
                             const int chunk = 2 * k + (mi >> 1);
@@ -943,10 +962,28 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                   (((chunk & 7) ^ (row & 7)) << 4);
                             uint32_t a0, a1, a2, a3;
                             ldsm_x4(addr, a0, a1, a2, a3);
+                            if constexpr (C::QSMEM) {
+                                if ((k & 1) == 0) {
+                                    // matrices: rows nt*8 .. +7 at d = 16k, 16k+8, 16k+16, 16k+24
+#pragma unroll
+                                    for (int nt = 0; nt < NT; ++nt)
+                                        ldsm_x4(qbase + (nt * 8 + (lane & 7)) * C::QROW +
+                                                    (16 * (k + (lane >> 4)) + 8 * ((lane >> 3) & 1)) * 2,
+                                                qb4[nt][0], qb4[nt][1], qb4[nt][2], qb4[nt][3]);
+                                }
+                            }
 #pragma unroll
                             for (int nt = 0; nt < NT; ++nt) {
-                                if (k & 1) mma_bf16(sac2[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
-                                else       mma_bf16(sacc[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
+                                uint32_t b0, b1;
+                                if constexpr (C::QSMEM) {
+                                    b0 = qb4[nt][(k & 1) * 2];
+                                    b1 = qb4[nt][(k & 1) * 2 + 1];
+                                } else {
+                                    b0 = qf[k][nt][0];
+                                    b1 = qf[k][nt][1];
+                                }
+                                if (k & 1) mma_bf16(sac2[nt], a0, a1, a2, a3, b0, b1);
+                                else       mma_bf16(sacc[nt], a0, a1, a2, a3, b0, b1);
                             }
                         }
                     } else {
@@ -1125,6 +1162,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_empty + 8 * slot);
+            }
+            if (C::QSMEM) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(seg_empty + 8 * qs);   // query rows read
             }
 
             // ---- finish the segment: merge the 4 warps' states -----------------
