@@ -233,13 +233,14 @@ def mode_step(args, w, pgd, dev, stream):
     ab = w.algorithmic_bytes()
 
     def decode(inp):
+        out = inp.get("out", m.out)
         if fused:
             pgd.decode_step(inp["q"], inp["kn"], inp["vn"], k, v, inp["bt"], inp["cl"],
                             w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, w.scale,
-                            m.out, max_context_len=mcl, k_scale=ks, v_scale=vs, stream=stream)
+                            out, max_context_len=mcl, k_scale=ks, v_scale=vs, stream=stream)
         else:
             pgd.paged_decode_attention(inp["q"], k, v, inp["bt"], inp["cl"], w.num_q_heads,
-                                       w.num_kv_heads, w.head_dim, w.block_size, w.scale, m.out,
+                                       w.num_kv_heads, w.head_dim, w.block_size, w.scale, out,
                                        max_context_len=mcl, k_scale=ks, v_scale=vs,
                                        stream=stream)
 
@@ -285,7 +286,8 @@ def mode_ex(args, w, pgd, dev, stream):
         if ev:
             ev[0].record(stream)
         pgd.paged_decode_attention_ex(inp["q"], k, v, inp["bt"], inp["cl"], w.num_q_heads,
-                                      w.num_kv_heads, w.head_dim, w.block_size, w.scale, m.out,
+                                      w.num_kv_heads, w.head_dim, w.block_size, w.scale,
+                                      inp.get("out", m.out),
                                       window=W, max_context_len=mcl, k_scale=ks, v_scale=vs,
                                       stream=stream)
         if ev:
@@ -336,8 +338,8 @@ def mode_kvp(args, w, pgd, dev, stream, rank, world):
         if ev:
             ev[1].record(stream)
         kvp.gather_partials(dec.o_local, dec.lse_local, dec.o_all, dec.lse_all)
-        pgd.merge_partials(dec.o_all, dec.lse_all, dec.out.view(rows, w.head_dim), dec.lse,
-                           stream=stream)
+        pgd.merge_partials(dec.o_all, dec.lse_all, inp.get("out", dec.out).view(rows, w.head_dim),
+                           dec.lse, stream=stream)
 
     bs, Hkv, D, e = w.block_size, w.num_kv_heads, w.head_dim, w.elem_bytes
     blocks = int(((length.astype(np.int64) + bs - 1) // bs).sum())
@@ -434,34 +436,71 @@ def run_ours(args, rank, world, local_rank):
     iso_ms = sum(a_.elapsed_time(b_) for a_, b_ in iso) / len(iso)
 
     # ---- end to end through the public API with host buffers ----------------
-    # every step copies its inputs from pinned host memory and reads the
-    # output back
-    dinp = {n: torch.empty_like(t) for n, t in m.inputs.items()}
-    hout = torch.empty(m.out.shape, dtype=m.out.dtype, pin_memory=True)
-    h2d_bytes = sum(h.numel() * h.element_size() for h in m.host.values())
-    d2h_bytes = hout.numel() * hout.element_size()
+    # Every step copies its inputs from pinned host memory (packed into one
+    # buffer, one copy) and reads its output back.  As in a serving loop, the
+    # input copy of step i+1 and the read-back of step i-1 run on their own
+    # streams while step i decodes (inputs and outputs double-buffered); all
+    # of every step's copies are inside the timed region.
+    names = list(m.host.keys())
+    nbytes = {n: m.host[n].numel() * m.host[n].element_size() for n in names}
+    offs, total = {}, 0
+    for n in names:
+        offs[n] = total
+        total += (nbytes[n] + 255) // 256 * 256
+    hpack = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+    for n in names:
+        hpack[offs[n]:offs[n] + nbytes[n]].copy_(m.host[n].reshape(-1).view(torch.uint8))
+    dpack = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(2)]
+    bufs = []
+    for b in range(2):
+        views = {n: dpack[b][offs[n]:offs[n] + nbytes[n]].view(m.host[n].dtype)
+                 .view(m.host[n].shape) for n in names}
+        views["out"] = torch.empty_like(m.out)
+        bufs.append(views)
+    hout = [torch.empty(m.out.shape, dtype=m.out.dtype, pin_memory=True) for _ in range(2)]
+    s_h2d = torch.cuda.Stream(device=dev)
+    s_d2h = torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of buffer b copied
+    ev_cmp = [torch.cuda.Event() for _ in range(2)]    # step using buffer b computed
+    ev_out = [torch.cuda.Event() for _ in range(2)]    # output of buffer b read back
+    h2d_bytes = total
+    d2h_bytes = hout[0].numel() * hout[0].element_size()
     Ke = max(1, min(K, args.e2e_steps))
 
-    def e2e_step():
-        for n, h in m.host.items():
-            dinp[n].copy_(h, non_blocking=True)
-        m.step(dinp)
-        hout.copy_(m.out, non_blocking=True)
+    def e2e_steps(n):
+        for i in range(n):
+            b = i % 2
+            if i >= 2:
+                s_h2d.wait_event(ev_cmp[b])            # step i-2 no longer reads buffer b
+            with torch.cuda.stream(s_h2d):
+                dpack[b].copy_(hpack, non_blocking=True)
+            ev_in[b].record(s_h2d)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])           # output of step i-2 read back
+            m.step(bufs[b])
+            ev_cmp[b].record(stream)
+            s_d2h.wait_event(ev_cmp[b])
+            with torch.cuda.stream(s_d2h):
+                hout[b].copy_(bufs[b]["out"], non_blocking=True)
+            ev_out[b].record(s_d2h)
 
-    for _ in range(3):
-        e2e_step()
+    e2e_steps(3)
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     f0 = torch.cuda.Event(enable_timing=True)
     f1 = torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(Ke):
-        e2e_step()
-    f1.record(stream)
+    f0.record(s_h2d)
+    e2e_steps(Ke)
+    s_d2h.wait_event(ev_cmp[(Ke - 1) % 2])
+    f1.record(s_d2h)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = f0.elapsed_time(f1) / Ke
+    # the kernels are deterministic: the read-back output is the resident run's
+    assert torch.equal(hout[(Ke - 1) % 2].view(torch.uint8), m.out.cpu().view(torch.uint8)), \
+        "end-to-end output differs from the device-resident run"
 
     # ---- aggregate over ranks ----------------------------------------------------
     ms_step = ms_total / K
@@ -513,7 +552,10 @@ def run_ours(args, rank, world, local_rank):
             "e2e": {"value": round(e2e_value, 1), "unit": "GB/s",
                     "us_per_step": round(e2e_ms * 1e3, 2),
                     "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
-                    "steps": Ke},
+                    "steps": Ke,
+                    "copies": "one packed H2D of the step's inputs and one D2H of its output "
+                              "per step, on their own streams, overlapping the neighbouring "
+                              "steps' decode (double-buffered)"},
             "gpu_launches": K * m.launches,
             "fused_step": m.fused,
             "clocks": clk,
