@@ -161,7 +161,9 @@ size_t pgd_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
  * all g query heads of its group, and keeps an online softmax; a sequence
  * whose tiles fall into several CTAs is merged by log-sum-exp by the CTA that
  * finishes its last share ("prefill and decode attention").  The result does
- * not depend on where the blocks sit in the pool.
+ * not depend on where the blocks sit in the pool, and repeated calls with the
+ * same inputs and grid give the same bits (the splits are merged in a fixed
+ * order).
  *
  *   q             device bf16 [num_seqs][num_q_heads][head_dim], 16-byte aligned
  *   k_cache, v_cache  device, HND layout, 16-byte aligned, num_blocks blocks

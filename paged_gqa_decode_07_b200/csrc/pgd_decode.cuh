@@ -8,40 +8,44 @@
 // with K_t / V_t read through the block table, and lse[s][i] its log-sum-exp.
 //
 // Work decomposition.  The batch is flattened into tiles (s, h, j): KV head h
-// of logical block j of sequence s, ordered by s, then h, then j.  The U tiles
-// are cut into G equal contiguous ranges, one per CTA, so every CTA streams
-// the same number of KV bytes whatever the length mix ("prefill and decode
-// attention": split along the KV length so that all SMs read at once).  Every
-// CTA derives the cut from context_lens itself (no host round trip).  Inside
-// its range a CTA walks "segments" (the part of one (s, h) unit that falls in
-// the range).  A segment that covers its whole unit writes `out` directly;
-// otherwise it writes a partial (o, lse) and the CTA that completes the
-// unit's last share merges the partials by log-sum-exp.
+// of logical block j of sequence s, ordered by s, then h, then j; each
+// (s, h) unit also weighs a fixed cost, so that a CTA given many short units
+// gets fewer of them.  The total is cut into G equal contiguous ranges, one
+// per CTA, so every CTA streams about the same KV bytes whatever the length
+// mix ("prefill and decode attention": split along the KV length so that all
+// SMs read at once).  Every CTA derives the cut from context_lens itself (no
+// host round trip).  Inside its range a CTA walks "segments" (the part of one
+// (s, h) unit that falls in the range).  A segment that covers its whole unit
+// writes `out` directly; otherwise it writes a partial (o, lse) and the CTA
+// that completes the unit's last share merges the partials by log-sum-exp.
 //
 // CTA = 4 consumer warps + 1 producer warp + 1 appender warp.  The producer
-// is the only warp that reads the inputs from global memory: it walks the
-// segments, writes a
+// is the only warp that reads the K/V inputs: it walks the segments, writes a
 // descriptor for each into a small shared-memory ring together with the
-// unit's query rows (bulk copy), loads the block-table entries 32 at a time,
-// and issues one TMA tensor load per (block, KV head) tile of K and of V into
-// a ring of 64-token stages (128-byte swizzle, mbarrier completion).  Each
-// K/V tile is fetched once and used by all g query heads of the group
-// ("prefill and decode attention": GQA reuse).  In a fused decode step the
-// appender warp writes each sequence's newest K/V row into the cache ahead of
-// the producer ("batching and attention" 3.4: the new token's slot), so the
-// append costs no extra launch.
+// unit's query rows (bulk copy), loads the block-table entries 32 at a time
+// (the next unit's while it issues the current one's tiles), and issues one
+// TMA tensor load per (block, KV head) tile of K and of V into a ring of
+// 64-token stages (128-byte swizzle, mbarrier completion).  Each K/V tile is
+// fetched once and used by all g query heads of the group ("prefill and
+// decode attention": GQA reuse).  In a fused decode step the appender warp
+// writes each sequence's newest K/V row into the cache ahead of the producer
+// ("batching and attention" 3.4: the new token's slot), so the append costs
+// no extra launch.
 //
-// Per stage the consumers run a small tensor-core contraction per warp
-// (mma.sync m16n8k16, fp32 accumulate) with the roles transposed so that the
-// group's query heads are the narrow N = 8 dimension:
-//   S^T[tokens][heads] = K[tokens][d] . Q^T[d][heads]   (each warp: 16 tokens)
-//   stage max per head through shared memory -> p = exp2(S - m)
-//   O^T[d][heads] += V^T[d][tokens] . P^T[tokens][heads] (each warp: D/4 dims)
-// which is the online softmax of "FlashAttention" applied stage by stage.
+// Consumer warp w owns tokens 16w .. 16w+15 of every stage and keeps its own
+// online softmax ("FlashAttention") over them, with a small tensor-core
+// contraction (mma.sync m16n8k16, fp32 accumulate) whose roles are
+// transposed so that the unit's query rows are the narrow N = 8 dimension:
+//   S^T[tokens][rows] = K[tokens][d] . Q^T[d][rows]
+//   row max over the warp's tokens (shuffles) -> p = exp2(S - m)
+//   P^T to the B-operand layout by a warp transpose (movmatrix)
+//   O^T[d][rows] += V^T[d][tokens] . P^T[tokens][rows]  (all of D)
+// The four warps' states are merged once per segment, in a fixed order.
 // With bf16 K/V the weights p enter the PV product as two bf16 terms,
 // p_hi = bf16(p) and p_lo = bf16(p - p_hi) (about 16 significant bits), and
 // the normaliser sums the fp32 p; with FP8 K/V they enter as f16 (11 bits)
-// and the normaliser sums those rounded values.
+// and the normaliser sums those rounded values.  A row's reference max moves
+// only when a score exceeds it by more than 2^8 (lazy rescaling).
 #pragma once
 
 #include "pgd_ptx.cuh"
