@@ -187,14 +187,17 @@ bool supported_block(int bs) { return bs == 16 || bs == 32 || bs == 64; }
 bool supported_group(int g) { return g >= 1 && g <= 16; }
 
 // Fixed cost of one (sequence, KV head) unit in a CTA (descriptor, query
-// rows, block-table fetch, first-tile latency, output) expressed as the K/V
-// bytes a CTA streams in the same time, about 2 us at 20 GB/s.  The batch is
-// cut by tiles + this many tile-equivalents per unit.
-constexpr long long kUnitOverheadBytes = 40 * 1024;
+// rows, block-table fetch, first-tile latency, merge, output) expressed as the
+// K/V bytes a CTA streams in the same time.  FP8 tiles take longer per byte
+// (the consumers convert every element), so the same time is fewer bytes.
+// The batch is cut by tiles + this many tile-equivalents per unit.
+constexpr long long kUnitOverheadBytes = 48 * 1024;
+constexpr long long kUnitOverheadBytesFp8 = 24 * 1024;
 
 int32_t unit_cost_tiles(int head_dim, int block_size, bool fp8) {
     const long long tile_kv = 2LL * block_size * head_dim * (fp8 ? 1 : 2);
-    return static_cast<int32_t>((kUnitOverheadBytes + tile_kv - 1) / tile_kv);
+    const long long unit = fp8 ? kUnitOverheadBytesFp8 : kUnitOverheadBytes;
+    return static_cast<int32_t>((unit + tile_kv - 1) / tile_kv);
 }
 
 }  // namespace
