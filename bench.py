@@ -87,6 +87,25 @@ def recorded_traffic(workload: str):
     return None
 
 
+def l2_replicas(read_bytes: int, cache_bytes: int, cap_bytes: int = 16 << 30) -> int:
+    """How many copies of the K/V caches the timed loop rotates through, one
+    per step, so that a cached row is read again only after at least 2x L2
+    of other K/V has streamed past it (1 when one step already reads that
+    much).  Capped so that the copies hold at most `cap_bytes`."""
+    if read_bytes >= 2 * L2_BYTES:
+        return 1
+    want = -(-2 * L2_BYTES // max(1, read_bytes))
+    return int(max(1, min(want, cap_bytes // max(1, cache_bytes))))
+
+
+def cache_copies(w, read_bytes, T):
+    """The caches (and FP8 scales) on the device, replicated per l2_replicas."""
+    R = l2_replicas(read_bytes, w.k_cache.nbytes + w.v_cache.nbytes)
+    ks = T(w.k_scale) if w.k_scale is not None else None
+    vs = T(w.v_scale) if w.v_scale is not None else None
+    return [(T(w.k_cache), T(w.v_cache)) for _ in range(R)], ks, vs
+
+
 def workload_desc(w) -> dict:
     return {"workload": f"{w.name}: {w.num_seqs} seqs, {w.num_tokens} context tokens "
                         f"(seed 0 draw), {w.num_q_heads} q / {w.num_kv_heads} kv heads, "
@@ -201,9 +220,9 @@ def _to_torch(a, dev=None, pin=False):
 
 
 class Mode:
-    """One kind of timed step.  step(inp, ev) runs one step on the tensors of
-    `inp` (device resident); with `ev` = (start, end) events it records them
-    around the dominant kernel's launch."""
+    """One kind of timed step.  step(inp, ev, r) runs one step on the tensors
+    of `inp` (device resident) and copy r of the caches; with `ev` = (start,
+    end) events it records them around the dominant kernel's launch."""
     single = True            # one launch per step: its duration = region / K
     kernel = "paged_decode_kernel"
     scaling = "weak"
@@ -211,6 +230,8 @@ class Mode:
     def __init__(self):
         self.inputs, self.host, self.out = {}, {}, None
         self.cfg = {}
+        self.replicas = 1
+        self.read_bytes = 0
 
 
 def mode_step(args, w, pgd, dev, stream):
@@ -218,9 +239,8 @@ def mode_step(args, w, pgd, dev, stream):
     the decode launch (pgd_decode_step), or --unfused: the two calls."""
     m = Mode()
     T = lambda a: _to_torch(a, dev)  # noqa: E731
-    k, v = T(w.k_cache), T(w.v_cache)
-    ks = T(w.k_scale) if w.k_scale is not None else None
-    vs = T(w.v_scale) if w.v_scale is not None else None
+    ab = w.algorithmic_bytes()
+    caches, ks, vs = cache_copies(w, ab["kv"], T)
     has_app = w.slot_mapping is not None
     arrays = {"q": w.q, "bt": w.block_table, "cl": w.context_lens}
     if has_app:
@@ -230,9 +250,8 @@ def mode_step(args, w, pgd, dev, stream):
     m.out = torch_empty_like(m.inputs["q"])
     fused = has_app and not args.unfused and len(w.slot_mapping) == w.num_seqs
     mcl = w.max_context_len
-    ab = w.algorithmic_bytes()
 
-    def decode(inp):
+    def decode(inp, k, v):
         out = inp.get("out", m.out)
         if fused:
             pgd.decode_step(inp["q"], inp["kn"], inp["vn"], k, v, inp["bt"], inp["cl"],
@@ -244,12 +263,13 @@ def mode_step(args, w, pgd, dev, stream):
                                        max_context_len=mcl, k_scale=ks, v_scale=vs,
                                        stream=stream)
 
-    def step(inp, ev=None):
+    def step(inp, ev=None, r=0):
+        k, v = caches[r]
         if has_app and not fused:
             pgd.kv_append(inp["kn"], inp["vn"], inp["sl"], k, v, stream=stream)
         if ev:
             ev[0].record(stream)
-        decode(inp)
+        decode(inp, k, v)
         if ev:
             ev[1].record(stream)
 
@@ -260,6 +280,7 @@ def mode_step(args, w, pgd, dev, stream):
     m.dec_bytes = ab["step_total"] if fused else ab["decode_total"]
     m.step_bytes = ab["step_total"]
     m.fused = fused
+    m.replicas, m.read_bytes = len(caches), ab["kv"]
     return m
 
 
@@ -270,19 +291,20 @@ def mode_ex(args, w, pgd, dev, stream):
     from workloads import multi_query
     m = Mode()
     T = lambda a: _to_torch(a, dev)  # noqa: E731
-    k, v = T(w.k_cache), T(w.v_cache)
-    ks = T(w.k_scale) if w.k_scale is not None else None
-    vs = T(w.v_scale) if w.v_scale is not None else None
-    if w.slot_mapping is not None:
-        pgd.kv_append(T(w.k_new), T(w.v_new), T(w.slot_mapping), k, v, stream=stream)
     L, W = args.q_len, args.window
+    ab = w.algorithmic_bytes(L, W)
+    caches, ks, vs = cache_copies(w, ab["kv"], T)
+    if w.slot_mapping is not None:
+        for k, v in caches:
+            pgd.kv_append(T(w.k_new), T(w.v_new), T(w.slot_mapping), k, v, stream=stream)
     arrays = {"q": multi_query(w, L, seed=0), "bt": w.block_table, "cl": w.context_lens}
     m.inputs = {n: T(a) for n, a in arrays.items()}
     m.host = {n: _to_torch(a, pin=True) for n, a in arrays.items()}
     m.out = torch_empty_like(m.inputs["q"])
     mcl = w.max_context_len
 
-    def step(inp, ev=None):
+    def step(inp, ev=None, r=0):
+        k, v = caches[r]
         if ev:
             ev[0].record(stream)
         pgd.paged_decode_attention_ex(inp["q"], k, v, inp["bt"], inp["cl"], w.num_q_heads,
@@ -293,8 +315,8 @@ def mode_ex(args, w, pgd, dev, stream):
         if ev:
             ev[1].record(stream)
 
-    ab = w.algorithmic_bytes(L, W)
     m.step, m.launches, m.fused = step, 1, False
+    m.replicas, m.read_bytes = len(caches), ab["kv"]
     m.kernel = f"paged_decode_kernel (q_len {L}, window {W})"
     m.dec_bytes = m.step_bytes = ab["decode_total"]
     m.cfg = {"q_len": L, "window": W, "visible_tokens":
@@ -314,10 +336,10 @@ def mode_kvp(args, w, pgd, dev, stream, rank, world):
     T = lambda a: _to_torch(a, dev)  # noqa: E731
     if w.slot_mapping is not None:
         raise SystemExit("--kvp needs a workload without an append payload")
-    k, v = T(w.k_cache), T(w.v_cache)
-    ks = T(w.k_scale) if w.k_scale is not None else None
-    vs = T(w.v_scale) if w.v_scale is not None else None
     start, length = kvp.plan(w.context_lens, w.block_size, world, rank)
+    bs, Hkv, D, e = w.block_size, w.num_kv_heads, w.head_dim, w.elem_bytes
+    slice_kv = int(length.astype(np.int64).sum()) * Hkv * D * 2 * e
+    caches, ks, vs = cache_copies(w, slice_kv, T)
     table = kvp.local_block_table(w.block_table, start, length, w.block_size)
     arrays = {"q": w.q, "bt": table, "cl": length}
     m.inputs = {n: T(a) for n, a in arrays.items()}
@@ -328,7 +350,8 @@ def mode_kvp(args, w, pgd, dev, stream, rank, world):
     mcl = int(length.max(initial=0))
     rows = w.num_seqs * w.num_q_heads
 
-    def step(inp, ev=None):
+    def step(inp, ev=None, r=0):
+        k, v = caches[r]
         if ev:
             ev[0].record(stream)
         pgd.paged_decode_partial(inp["q"], k, v, inp["bt"], inp["cl"], w.num_q_heads,
@@ -341,9 +364,7 @@ def mode_kvp(args, w, pgd, dev, stream, rank, world):
         pgd.merge_partials(dec.o_all, dec.lse_all, inp.get("out", dec.out).view(rows, w.head_dim),
                            dec.lse, stream=stream)
 
-    bs, Hkv, D, e = w.block_size, w.num_kv_heads, w.head_dim, w.elem_bytes
     blocks = int(((length.astype(np.int64) + bs - 1) // bs).sum())
-    slice_kv = int(length.astype(np.int64).sum()) * Hkv * D * 2 * e
     meta = blocks * 4 + w.num_seqs * 4 + (2 * Hkv * 4 if w.kv_dtype == "e4m3" else 0)
     # the slice kernel reads q, its slice and metadata, and writes fp32 o + lse
     m.dec_bytes = slice_kv + meta + rows * D * 2 + rows * (D + 1) * 4
@@ -353,6 +374,7 @@ def mode_kvp(args, w, pgd, dev, stream, rank, world):
     m.step, m.single, m.launches, m.fused = step, False, 2, False
     m.kernel = "paged_decode_kernel (fp32 split result of the rank's KV slice)"
     m.scaling = "strong"
+    m.replicas, m.read_bytes = len(caches), slice_kv
     m.cfg = {"kvp_ranks": world, "exchange_bytes_per_rank": dec.exchange_bytes(),
              "slice_tokens_this_rank": int(length.sum())}
     return m
@@ -392,8 +414,9 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
 
     # ---- warm-up -------------------------------------------------------------
-    for _ in range(args.warmup):
-        m.step(m.inputs)
+    R = m.replicas
+    for i in range(max(args.warmup, R)):
+        m.step(m.inputs, None, i % R)
     torch.cuda.synchronize()
     assert pgd.get_device_error() == 0
 
@@ -415,7 +438,7 @@ def run_ours(args, rank, world, local_rank):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(K):
-        m.step(m.inputs, None if m.single else ev_dec[i])
+        m.step(m.inputs, None if m.single else ev_dec[i], i % R)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -430,8 +453,8 @@ def run_ours(args, rank, world, local_rank):
     # for reference: the dominant launch bracketed by its own events, one at a time
     iso = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(min(K, 50))]
-    for ev in iso:
-        m.step(m.inputs, ev)
+    for i, ev in enumerate(iso):
+        m.step(m.inputs, ev, i % R)
     torch.cuda.synchronize()
     iso_ms = sum(a_.elapsed_time(b_) for a_, b_ in iso) / len(iso)
 
@@ -478,7 +501,7 @@ def run_ours(args, rank, world, local_rank):
             stream.wait_event(ev_in[b])
             if i >= 2:
                 stream.wait_event(ev_out[b])           # output of step i-2 read back
-            m.step(bufs[b])
+            m.step(bufs[b], None, i % R)
             ev_cmp[b].record(stream)
             s_d2h.wait_event(ev_cmp[b])
             with torch.cuda.stream(s_d2h):
@@ -520,12 +543,18 @@ def run_ours(args, rank, world, local_rank):
         cfg.update(m.cfg)
         if args.math != "tensor_core":
             cfg["math"] = args.math
-        kv_mb = w.algorithmic_bytes(max(1, args.q_len), args.window)["kv"] / 1e6
+        kv_mb = m.read_bytes / 1e6
+        if R == 1:
+            l2 = (f"inputs larger than L2 ({kv_mb:.0f} MB of KV read per step vs "
+                  f"{L2_BYTES / 2**20:.0f} MiB L2); no flush")
+        else:
+            l2 = (f"{kv_mb:.0f} MB of KV read per step is under 2x the {L2_BYTES / 2**20:.0f} "
+                  f"MiB L2: the steps rotate through {R} copies of the caches, so "
+                  f"{R * kv_mb:.0f} MB of KV streams between two reads of a row; no flush")
         cfg.update({"parallelism": (f"KV parallel over {world} rank(s) (one batch, each "
                                     f"sequence split along its length)") if args.kvp else
                     f"replicas x{world} (independent batch per GPU)",
-                    "l2": f"inputs larger than L2 ({kv_mb:.0f} MB of KV read per step "
-                          f"vs {L2_BYTES / 2**20:.0f} MiB L2); no flush",
+                    "l2": l2, "cache_copies": R,
                     "global_batch": w.num_seqs * (1 if args.kvp else world)})
         default_mode = not args.kvp and args.q_len == 1 and args.window == 0
         line = {
