@@ -27,7 +27,7 @@ constexpr int kMaxDevices = 64;
 constexpr int kMaxCtasPerSmForSizing = 4;
 
 struct DeviceState {
-    bool init = false;
+    std::atomic<bool> init{false};   // set once, after the fields below
     int sms = 0;
     uint32_t *flags = nullptr;
     void *ws = nullptr;        // library-owned decode workspace (split partials)
@@ -45,15 +45,15 @@ pgd_status device_state(DeviceState **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PGD_ERR_CUDA;
     DeviceState &d = g_dev[dev];
-    if (!d.init) {
+    if (!d.init.load(std::memory_order_acquire)) {
         std::lock_guard<std::mutex> lk(g_mu);
-        if (!d.init) {
+        if (!d.init.load(std::memory_order_relaxed)) {
             if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
                 return PGD_ERR_CUDA;
             void *p = nullptr;
             if (cudaGetSymbolAddress(&p, g_flags) != cudaSuccess) return PGD_ERR_CUDA;
             d.flags = static_cast<uint32_t *>(p);
-            d.init = true;
+            d.init.store(true, std::memory_order_release);
         }
     }
     *out = &d;
@@ -607,7 +607,7 @@ constexpr size_t kStaticCounterBytes = sizeof(int32_t) * kStaticMaxUnits;
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 struct StaticScratch {
-    bool ready = false;
+    std::atomic<bool> ready{false};   // set once, after ptr
     unsigned char *ptr = nullptr;   // device address of g_static_scratch
 };
 StaticScratch g_static[kMaxDevices];
@@ -619,13 +619,13 @@ pgd_status static_scratch(unsigned char **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PGD_ERR_CUDA;
     StaticScratch &s = g_static[dev];
-    if (!s.ready) {
+    if (!s.ready.load(std::memory_order_acquire)) {
         std::lock_guard<std::mutex> lk(g_mu);
-        if (!s.ready) {
+        if (!s.ready.load(std::memory_order_relaxed)) {
             void *p = nullptr;
             if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return PGD_ERR_CUDA;
             s.ptr = static_cast<unsigned char *>(p);
-            s.ready = true;
+            s.ready.store(true, std::memory_order_release);
         }
     }
     *out = s.ptr;
