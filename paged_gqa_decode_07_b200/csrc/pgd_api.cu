@@ -200,6 +200,24 @@ int32_t unit_cost_tiles(int head_dim, int block_size, bool fp8) {
     return static_cast<int32_t>((unit + tile_kv - 1) / tile_kv);
 }
 
+// Automatic grid: one wave of resident CTAs (sms x occ), fewer for small
+// batches (at least 4 stages of tiles per CTA).  With fewer (sequence, KV
+// head) units than CTAs, the grid is rounded down to a multiple of the unit
+// count when that drops at most 1/16 of it: with units of equal length every
+// CTA then holds one piece of one unit instead of the ends of two.
+long long auto_grid(int sms, int occ, int32_t num_seqs, int32_t num_kv_heads,
+                    int32_t max_blocks_per_seq, int32_t block_size, int32_t max_context_len) {
+    long long grid = static_cast<long long>(sms) * occ;
+    const long long units = static_cast<long long>(num_seqs) * num_kv_heads;
+    if (units > 0 && units < grid && grid % units <= grid / 16) grid -= grid % units;
+    const long long cap_tokens = static_cast<long long>(max_blocks_per_seq) * block_size;
+    const long long max_ctx =
+        max_context_len > 0 ? std::min<long long>(max_context_len, cap_tokens) : cap_tokens;
+    const long long tiles_upper = units * ((max_ctx + block_size - 1) / block_size);
+    const long long min_tiles = 4 * (kStageTokens / block_size);   // >= 4 stages per CTA
+    return std::max(1LL, std::min(grid, (tiles_upper + min_tiles - 1) / min_tiles));
+}
+
 }  // namespace
 
 extern "C" {
@@ -339,14 +357,8 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     if (grid == 0) {
         const int occ = var.occ();
         if (occ <= 0) return PGD_ERR_CUDA;
-        grid = static_cast<long long>(d->sms) * occ;
-        const long long cap_tokens = static_cast<long long>(max_blocks_per_seq) * block_size;
-        const long long max_ctx =
-            max_context_len > 0 ? std::min<long long>(max_context_len, cap_tokens) : cap_tokens;
-        const long long tiles_upper =
-            static_cast<long long>(num_seqs) * num_kv_heads * ((max_ctx + block_size - 1) / block_size);
-        const long long min_tiles = 4 * (kStageTokens / block_size);   // >= 4 stages per CTA
-        grid = std::max(1LL, std::min(grid, (tiles_upper + min_tiles - 1) / min_tiles));
+        grid = auto_grid(d->sms, occ, num_seqs, num_kv_heads, max_blocks_per_seq, block_size,
+                         max_context_len);
     }
     if (grid > (1LL << 24)) return PGD_ERR_INVALID_ARG;
 
@@ -683,14 +695,8 @@ extern "C" pgd_status pgd_paged_decode_attention_noalloc(
     if (grid == 0) {
         const int occ = var.occ();
         if (occ <= 0) return PGD_ERR_CUDA;
-        grid = static_cast<long long>(d->sms) * occ;
-        const long long cap_tokens = static_cast<long long>(max_blocks_per_seq) * block_size;
-        const long long max_ctx =
-            max_context_len > 0 ? std::min<long long>(max_context_len, cap_tokens) : cap_tokens;
-        const long long tiles_upper =
-            static_cast<long long>(num_seqs) * num_kv_heads * ((max_ctx + block_size - 1) / block_size);
-        const long long min_tiles = 4 * (kStageTokens / block_size);
-        grid = std::max(1LL, std::min(grid, (tiles_upper + min_tiles - 1) / min_tiles));
+        grid = auto_grid(d->sms, occ, num_seqs, num_kv_heads, max_blocks_per_seq, block_size,
+                         max_context_len);
         while (grid > 1 && ws_layout(g, head_dim, grid).total > avail) --grid;
     }
     if (grid > (1LL << 24)) return PGD_ERR_INVALID_ARG;
