@@ -106,6 +106,30 @@ def cache_copies(w, read_bytes, T):
     return [(T(w.k_cache), T(w.v_cache)) for _ in range(R)], ks, vs
 
 
+def copy_probe(dev, nbytes: int = 2 << 30, reps: int = 20) -> dict:
+    """HBM copy bandwidth in this process: the best of `reps` device-to-device
+    copies of an `nbytes` buffer, counting the bytes read and written."""
+    import torch
+    src = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    dst = torch.empty_like(src)
+    src.fill_(1)
+    for _ in range(3):
+        dst.copy_(src)
+    best = float("inf")
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dst.copy_(src)
+        b.record()
+        b.synchronize()
+        best = min(best, a.elapsed_time(b))
+    del src, dst
+    torch.cuda.empty_cache()
+    return {"gbs": round(2 * nbytes / (best * 1e-3) / 1e9, 1), "bytes_per_copy": 2 * nbytes,
+            "how": f"best of {reps} device-to-device copies of {nbytes >> 30} GiB "
+                   "(read + write bytes), same process, after the timed regions"}
+
+
 def workload_desc(w) -> dict:
     return {"workload": f"{w.name}: {w.num_seqs} seqs, {w.num_tokens} context tokens "
                         f"(seed 0 draw), {w.num_q_heads} q / {w.num_kv_heads} kv heads, "
@@ -534,6 +558,7 @@ def run_ours(args, rank, world, local_rank):
     # the dominant kernel of this rank (rank 0 prints its own launch figures)
     achieved = m.dec_bytes / (dec_avg_ms * 1e-3) / 1e9
 
+    probe = copy_probe(dev)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.cpu_seconds)
@@ -566,6 +591,8 @@ def run_ours(args, rank, world, local_rank):
             "config": cfg,
             "pct_of_measured_hbm": round(100 * value / world / peak, 1),
             "pct_of_nominal_8tbs": round(100 * value / world / 8000.0, 1),
+            "pct_of_same_run_copy": round(100 * achieved / probe["gbs"], 1),
+            "copy_probe": probe,
             "roofline": {"bound": "hbm", "kernel": m.kernel,
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
