@@ -191,8 +191,13 @@ size_t pgd_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
  *                 its own zeroed device buffer (grown the same way).  Calls
  *                 that share a workspace, or run on one device at the same
  *                 time, must not overlap on the GPU.
- *   num_ctas      0 = automatic grid (a multiple of the SM count); > 0 forces
- *                 that many CTAs (used to test split-count invariance)
+ *   num_ctas      0 = automatic grid: one wave of resident CTAs (SM count x
+ *                 CTAs per SM); with fewer (sequence, KV head) units than
+ *                 that, rounded down to a multiple of the unit count when
+ *                 this drops at most 1/16 of the wave; fewer for small
+ *                 batches (at least four 64-token stages of tiles per CTA,
+ *                 from max_context_len).  > 0 forces that many CTAs (used
+ *                 to test split-count invariance)
  *   stream        cudaStream_t as void*
  */
 pgd_status pgd_paged_decode_attention(
