@@ -65,3 +65,24 @@ def test_append_payload_bytes():
     n = len(w.slot_mapping)
     # k_new and v_new read, the same rows written into the caches, the slots read
     assert w.algorithmic_bytes()["append"] == 4 * n * 2 * 128 * 2 + 8 * n
+
+
+def _bench_args_rc(*args):
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), *args],
+                       capture_output=True, text=True, timeout=120)
+    return r.returncode, r.stderr
+
+
+def test_bench_rejects_too_few_warmup_steps():
+    rc, err = _bench_args_rc("--warmup", "2")
+    assert rc == 2 and "warmup" in err
+
+
+def test_bench_rejects_kvp_with_other_rows():
+    for extra in (["--q-len", "2"], ["--window", "64"], ["--unfused"]):
+        rc, err = _bench_args_rc("--kvp", *extra)
+        assert rc == 2 and "kvp" in err, extra
