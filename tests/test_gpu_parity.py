@@ -192,6 +192,20 @@ def test_full_size_sampled(name):
     if w.slot_mapping is not None:
         ek, ev = oracle_caches(w)
         assert np.array_equal(host_bits(d.k), ek) and np.array_equal(host_bits(d.v), ev)
+        # the launch the decode-step benchmark times: append fused into the
+        # decode (pgd_decode_step), same bits as the two launches above
+        from tests.gpu_helpers import dev_cache
+        kn, vn = _step_payload(w)
+        d2 = Dev(w)
+        lse2 = torch.empty_like(lse)
+        out2 = pgd.decode_step(d2.q, dev_cache(kn), dev_cache(vn), d2.k, d2.v, d2.bt, d2.cl,
+                               w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
+                               w.scale, max_context_len=w.max_context_len, k_scale=d2.ks,
+                               v_scale=d2.vs, lse_out=lse2)
+        torch.cuda.synchronize()
+        assert torch.equal(out2.view(torch.int16), out.view(torch.int16))
+        assert torch.equal(lse2, lse)
+        assert np.array_equal(host_bits(d2.k), ek) and np.array_equal(host_bits(d2.v), ev)
 
 
 # --------------------------------------------------------------------------- #
