@@ -254,13 +254,15 @@ pgd_status pgd_decode_step(
  *   q        device bf16 [num_seqs][q_len][num_q_heads][head_dim]
  *   out      device bf16 [num_seqs][q_len][num_q_heads][head_dim]
  *   lse_out  optional fp32 [num_seqs][q_len][num_q_heads]
- *   q_len    >= 1 with g * q_len <= 16 (g = num_q_heads / num_kv_heads): every
+ *   q_len    >= 1 with g * q_len <= 32 (g = num_q_heads / num_kv_heads): every
  *            query row of a KV head rides on one pass over its K/V tiles
+ *            (up to 16 rows all four consumer warps hold every row; 17 to 32
+ *            rows are split into two groups of 16, each over all tokens)
  *   window   0 = the whole causal range; > 0 = the last `window` positions
  *   workspace  at least pgd_decode_workspace_bytes(num_seqs,
  *            num_q_heads * q_len, num_kv_heads, head_dim) bytes, or NULL/0
  *   all other arguments and errors as pgd_paged_decode_attention; q_len = 1,
- *   window = 0 gives exactly that call.  g * q_len > 16 returns
+ *   window = 0 gives exactly that call.  g * q_len > 32 returns
  *   PGD_ERR_UNSUPPORTED.  Blocks that lie wholly before a window are not read.
  */
 pgd_status pgd_paged_decode_attention_ex(
@@ -299,6 +301,27 @@ typedef enum {
 
 pgd_status pgd_set_decode_math(pgd_decode_math math);
 pgd_decode_math pgd_get_decode_math(void);
+
+/* ------------------------------------------------------------------------ */
+/* Test hook for the timeout path                                           */
+/* ------------------------------------------------------------------------ */
+/*
+ * Every wait inside the decode kernels (a K/V stage landing, a segment
+ * descriptor, a free ring slot, an appended row) is bounded: after the limit
+ * the kernel raises the timeout flag (8), its warps leave together, the
+ * producer still waits for every copy it issued (with its own fixed limit of
+ * 0.2 s) so nothing lands after the CTA exits, and pgd_get_device_error()
+ * returns PGD_ERR_TIMEOUT and re-zeroes the arrival counters, so the next
+ * call starts clean.  No correct input makes a wait run out, so this hook
+ * exists to test that path: a limit of a few ns makes the waits give up.
+ *
+ * pgd_debug_set_wait_limit_ns -- process-wide limit of those waits for the
+ * decode launches that follow, in ns; 0 restores the default (1 s).  Outputs
+ * of a launch that timed out are undefined.  Not for production use.
+ * pgd_debug_get_wait_limit_ns -- the current limit.
+ */
+pgd_status pgd_debug_set_wait_limit_ns(uint64_t limit_ns);
+uint64_t pgd_debug_get_wait_limit_ns(void);
 
 /* ------------------------------------------------------------------------ */
 /* KV parallelism: one sequence's KV split along its length over GPUs       */
@@ -363,10 +386,13 @@ pgd_status pgd_paged_decode_partial(
  *
  * Arguments are those of pgd_paged_decode_attention without the workspace:
  * the caller still provides every input and output.  The split partials and
- * the arrival counters live in one static device array of 8 MiB per device
- * (held by every GPU that loads the library until the process exits).  The
- * call allocates nothing: no cudaMalloc, no cudaFree, no allocating library
- * routine.
+ * the arrival counters live in one static device array of 8 MiB per device,
+ * held until the process exits.  With CUDA's default lazy module loading the
+ * array is committed on a device at the first call of this library there
+ * (any entry point), not when the library is loaded: make one call on each
+ * device before reserving the KV-cache pool, so that the 8 MiB are already
+ * taken.  The call allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library routine.
  *   - Limits: num_seqs * num_kv_heads <= 65536, and the split partials of the
  *     grid must fit in the rest of the array; an automatic grid is reduced to
  *     fit, an explicit num_ctas that does not fit is rejected.  Requests past

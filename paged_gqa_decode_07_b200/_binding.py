@@ -72,6 +72,10 @@ def load_library():
     lib.pgd_set_decode_math.argtypes = [st]
     lib.pgd_get_decode_math.restype = st
     lib.pgd_get_decode_math.argtypes = []
+    lib.pgd_debug_set_wait_limit_ns.restype = st
+    lib.pgd_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.pgd_debug_get_wait_limit_ns.restype = ctypes.c_uint64
+    lib.pgd_debug_get_wait_limit_ns.argtypes = []
     lib.pgd_kvp_plan.restype = st
     lib.pgd_kvp_plan.argtypes = [P, i32, i32, i32, i32, P, P]
     lib.pgd_decode_step.restype = st
@@ -336,6 +340,18 @@ def set_decode_math(math: str) -> None:
 def get_decode_math() -> str:
     v = int(load_library().pgd_get_decode_math())
     return {b: a for a, b in _MATH.items()}[v]
+
+
+def debug_set_wait_limit_ns(limit_ns: int) -> None:
+    """Limit of the decode kernels' pipeline waits, in ns, for the launches
+    that follow (pgd_debug_set_wait_limit_ns); 0 restores the default 1 s.
+    A test hook for the timeout path."""
+    _check(load_library().pgd_debug_set_wait_limit_ns(int(limit_ns)),
+           "pgd_debug_set_wait_limit_ns")
+
+
+def debug_get_wait_limit_ns() -> int:
+    return int(load_library().pgd_debug_get_wait_limit_ns())
 
 
 def kvp_plan(context_lens, block_size: int, world_size: int, rank: int):

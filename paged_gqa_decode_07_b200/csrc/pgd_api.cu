@@ -97,6 +97,46 @@ pgd_status encode_kv_map(CUtensorMap *m, const void *base, int D, int E, int bs,
     return r == CUDA_SUCCESS ? PGD_OK : PGD_ERR_CUDA;
 }
 
+// Encoding a tensor map costs a driver call on the host, and a serving loop
+// passes the same caches on every step, so each host thread keeps the maps it
+// encoded last.  A map holds only the address, shape and strides it was
+// encoded from, so an entry with the same key is the same map whatever
+// happened to the memory in between.
+struct KvMapKey {
+    const void *base;
+    long long rows;
+    int D, E, bs;
+    bool operator==(const KvMapKey &o) const {
+        return base == o.base && rows == o.rows && D == o.D && E == o.E && bs == o.bs;
+    }
+};
+
+pgd_status cached_kv_map(CUtensorMap *m, const void *base, int D, int E, int bs,
+                         long long rows) {
+    constexpr int kEntries = 8;
+    struct Entry {
+        KvMapKey key;
+        CUtensorMap map;
+        bool used;
+    };
+    thread_local Entry cache[kEntries] = {};
+    thread_local int next = 0;
+    const KvMapKey key{base, rows, D, E, bs};
+    for (const Entry &e : cache)
+        if (e.used && e.key == key) {
+            *m = e.map;
+            return PGD_OK;
+        }
+    const pgd_status st = encode_kv_map(m, base, D, E, bs, rows);
+    if (st != PGD_OK) return st;
+    Entry &e = cache[next];
+    next = (next + 1) % kEntries;
+    e.key = key;
+    e.map = *m;
+    e.used = true;
+    return PGD_OK;
+}
+
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -156,12 +196,16 @@ bool pick_bs(int bs, int nt, Variant *v) {
     }
     PGD_CASE(16, 1) PGD_CASE(32, 1) PGD_CASE(64, 1)
     PGD_CASE(16, 2) PGD_CASE(32, 2) PGD_CASE(64, 2)
+    PGD_CASE(16, 4) PGD_CASE(32, 4) PGD_CASE(64, 4)
 #undef PGD_CASE
     return false;
 }
 
 // Consumer math of the decode kernels (pgd_set_decode_math); process-wide.
 std::atomic<int> g_math{PGD_MATH_TENSOR_CORE};
+
+// Limit of the decode kernels' pipeline waits in ns (pgd_debug_set_wait_limit_ns).
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
 
 template <int CC>
 bool pick_cuda_core(int bs, Variant *v) {
@@ -328,7 +372,7 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     if (head_dim != 128 && head_dim != 256) return PGD_ERR_UNSUPPORTED;
     if (fp8 && head_dim != 128) return PGD_ERR_UNSUPPORTED;
     const int rows = g * q_len;                 // query rows per (sequence, KV head)
-    if (rows > 16) return PGD_ERR_UNSUPPORTED;
+    if (rows > 32) return PGD_ERR_UNSUPPORTED;
     if (static_cast<long long>(num_blocks) * num_kv_heads >= INT_MAX ||
         static_cast<long long>(max_blocks_per_seq) * block_size >= INT_MAX)
         return PGD_ERR_UNSUPPORTED;
@@ -348,7 +392,7 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     DeviceState *d = nullptr;
     pgd_status st = device_state(&d);
     if (st != PGD_OK) return st;
-    const int nt = rows > 8 ? 2 : 1;
+    const int nt = rows > 16 ? 4 : rows > 8 ? 2 : 1;   // n-tiles of 8 query rows
     Variant var;
     if (!pick_variant(head_dim, block_size, nt, fp8, rows, &var)) return PGD_ERR_UNSUPPORTED;
 
@@ -394,8 +438,8 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     std::memset(&a, 0, sizeof(a));
     const int E = fp8 ? 1 : 2;
     const long long kv_rows = static_cast<long long>(num_blocks) * num_kv_heads;
-    if ((st = encode_kv_map(&a.tmK, k_cache, head_dim, E, block_size, kv_rows)) != PGD_OK) return st;
-    if ((st = encode_kv_map(&a.tmV, v_cache, head_dim, E, block_size, kv_rows)) != PGD_OK) return st;
+    if ((st = cached_kv_map(&a.tmK, k_cache, head_dim, E, block_size, kv_rows)) != PGD_OK) return st;
+    if ((st = cached_kv_map(&a.tmV, v_cache, head_dim, E, block_size, kv_rows)) != PGD_OK) return st;
     DecodeParams &p = a.p;
     p.q = static_cast<const uint16_t *>(q);
     p.out = static_cast<uint16_t *>(out);
@@ -424,6 +468,7 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     p.window = window;
     p.rows = rows;
     p.out_f32 = out_f32 ? 1 : 0;
+    p.wait_ns = g_wait_ns.load();
     a.grid = static_cast<int>(grid);
     a.stream = s;
     cudaError_t e = var.launch(a);
@@ -499,6 +544,13 @@ pgd_status pgd_set_decode_math(pgd_decode_math math) {
 pgd_decode_math pgd_get_decode_math(void) {
     return static_cast<pgd_decode_math>(g_math.load());
 }
+
+pgd_status pgd_debug_set_wait_limit_ns(uint64_t limit_ns) {
+    g_wait_ns.store(limit_ns == 0 ? kDefaultWaitNs : limit_ns);
+    return PGD_OK;
+}
+
+uint64_t pgd_debug_get_wait_limit_ns(void) { return g_wait_ns.load(); }
 
 pgd_status pgd_kvp_plan(const int32_t *context_lens, int32_t num_seqs, int32_t block_size,
                         int32_t world_size, int32_t rank, int32_t *block_start,
@@ -688,8 +740,12 @@ extern "C" pgd_status pgd_paged_decode_attention_noalloc(
     Variant var;
     if (!pick_variant(head_dim, block_size, nt, fp8, g, &var)) return PGD_ERR_UNSUPPORTED;
 
-    // grid: as the allocating entry point, then capped so that the split
-    // partials fit behind the counters in the static array
+    // grid: as the allocating entry point, capped so that the split partials
+    // fit behind the counters in the static array.  A CTA's partials take
+    // 8 * g * (head_dim + 1) bytes (two fp32 slots of g rows), so the array
+    // holds the partials of at least 247 CTAs (g 16, head_dim 256) and of
+    // 484 at head_dim 128: more than one wave of the automatic grid on a
+    // 148-SM B200, where the cap never applies.
     const size_t avail = kStaticScratchBytes - kStaticCounterBytes;
     long long grid = num_ctas;
     if (grid == 0) {
@@ -697,7 +753,12 @@ extern "C" pgd_status pgd_paged_decode_attention_noalloc(
         if (occ <= 0) return PGD_ERR_CUDA;
         grid = auto_grid(d->sms, occ, num_seqs, num_kv_heads, max_blocks_per_seq, block_size,
                          max_context_len);
-        while (grid > 1 && ws_layout(g, head_dim, grid).total > avail) --grid;
+        const long long per_cta = 8LL * g * (head_dim + 1);
+        const long long fit = std::max(1LL, static_cast<long long>(avail - 512) / per_cta);
+        if (grid > fit) {
+            grid = fit;
+            if (units < grid && grid % units <= grid / 16) grid -= grid % units;
+        }
     }
     if (grid > (1LL << 24)) return PGD_ERR_INVALID_ARG;
     const WsLayout lay = ws_layout(g, head_dim, grid);
@@ -712,8 +773,8 @@ extern "C" pgd_status pgd_paged_decode_attention_noalloc(
     std::memset(&a, 0, sizeof(a));
     const int E = fp8 ? 1 : 2;
     const long long rows = static_cast<long long>(num_blocks) * num_kv_heads;
-    if ((st = encode_kv_map(&a.tmK, k_cache, head_dim, E, block_size, rows)) != PGD_OK) return st;
-    if ((st = encode_kv_map(&a.tmV, v_cache, head_dim, E, block_size, rows)) != PGD_OK) return st;
+    if ((st = cached_kv_map(&a.tmK, k_cache, head_dim, E, block_size, rows)) != PGD_OK) return st;
+    if ((st = cached_kv_map(&a.tmV, v_cache, head_dim, E, block_size, rows)) != PGD_OK) return st;
     uint8_t *parts = scratch + kStaticCounterBytes;
     DecodeParams &p = a.p;
     p.q = static_cast<const uint16_t *>(q);
@@ -738,6 +799,7 @@ extern "C" pgd_status pgd_paged_decode_attention_noalloc(
     p.q_len = 1;
     p.window = 0;
     p.rows = g;
+    p.wait_ns = g_wait_ns.load();
     a.grid = static_cast<int>(grid);
     a.stream = s;
     e = var.launch(a);

@@ -83,6 +83,9 @@ struct DecodeParams {
     // 1: out holds fp32 values (the unrounded split result a caller merges
     // with other splits of the same rows); 0: bf16
     int32_t out_f32;
+    // limit of every pipeline wait in ns (kDefaultWaitNs unless a test of
+    // the timeout path shortens it)
+    uint64_t wait_ns;
 };
 
 constexpr int kConsumerWarps = 4;
@@ -108,6 +111,10 @@ struct SegDesc {
 // CC = 0: tensor-core (mma.sync) consumers; CC = 4 or 8: the CUDA-core
 // variant (FMA dot products with warp-shuffle reductions) for up to CC query
 // rows, kept to compare the two on this bandwidth-bound path.
+// NT = n-tiles of 8 query rows per unit: 1 (up to 8 rows), 2 (16) or 4 (32).
+// With NT = 4 the consumer warps split into two row groups of 16 rows (warps
+// 0, 1 and 2, 3) and each warp takes 32 tokens of every stage, so a stage is
+// still read once for all 32 rows.
 template <int D, int BS, int NT, bool FP8, int NSTAGES, int CC = 0>
 struct DecodeCfg {
     static constexpr int E = FP8 ? 1 : 2;                // bytes per KV element
@@ -117,6 +124,10 @@ struct DecodeCfg {
     static constexpr int BPS = kStageTokens / BS;        // blocks per stage
     static constexpr int STAGE_KV = BPS * TILE;          // K (or V) bytes per stage
     static constexpr int STAGE = 2 * STAGE_KV;
+    static constexpr int RG = NT == 4 ? 2 : 1;           // row groups of consumer warps
+    static constexpr int NTW = NT / RG;                  // n-tiles each warp holds
+    static constexpr int GW = kConsumerWarps / RG;       // warps per row group
+    static constexpr int SUBS = RG;                      // 16-token sub-tiles per warp and stage
     static constexpr int NP = 8 * NT;                    // padded query rows per unit
     static constexpr int DT = D / 16;                    // PV m-tiles (each warp: all of D)
     static constexpr int KSTEPS = D / 16;                // QK k-steps
@@ -126,14 +137,16 @@ struct DecodeCfg {
     static constexpr bool QSMEM = D == 256 && !FP8 && CC == 0;
     static constexpr int QROW = QSMEM ? D * 2 + 16 : D * 2;
     static constexpr int QSLOT = NP * QROW;              // query rows of one unit
-    // descriptor ring depth (one slot for 16 query rows at head_dim 128, so
-    // that two CTAs still fit on an SM)
-    static constexpr int NSEG = CC ? 2 : (D == 128 ? (QSLOT >= 4096 ? 1 : 3) : 2);
+    // descriptor ring depth (one slot for 16 or more query rows at head_dim
+    // 128, so that two CTAs still fit on an SM; one for 32 rows at 256)
+    static constexpr int NSEG =
+        CC ? 2 : (NT == 4 ? 1 : (D == 128 ? (QSLOT >= 4096 ? 1 : 3) : 2));
     static constexpr int OROW = D + 4;                   // sO row stride in floats
     // shared memory carve-up (offsets from a 1024-aligned base)
-    static constexpr int OFF_O = NSTAGES * STAGE;        // two 8-row O buffers
+    static constexpr int OFF_O = NSTAGES * STAGE;        // 8-row O merge buffers
     static constexpr int OBUF = 8 * OROW * 4;
-    static constexpr int OFF_Q = OFF_O + 2 * OBUF;
+    static constexpr int NOBUF = RG == 1 ? 2 : 1;        // A and B, or one per round
+    static constexpr int OFF_Q = OFF_O + NOBUF * OBUF;
     static constexpr int OFF_SEG = OFF_Q + NSEG * QSLOT;
     static constexpr int OFF_RED = OFF_SEG + NSEG * (int)sizeof(SegDesc);   // warps' row max
     static constexpr int OFF_LSUM = OFF_RED + kConsumerWarps * NP * 4;      // warps' row sum
@@ -154,6 +167,7 @@ struct DecodeCfg {
     static_assert(sizeof(SegDesc) % 16 == 0, "descriptor alignment");
     static_assert(OFF_Q % 16 == 0, "bulk copies need 16-byte aligned destinations");
     static_assert(D != 128 || SMEM <= 113 * 1024, "two CTAs per SM at head_dim 128");
+    static_assert(SMEM <= 227 * 1024, "shared memory of one CTA");
 };
 
 struct Misc {                 // CTA-wide scalars in shared memory
@@ -326,17 +340,18 @@ __device__ __forceinline__ long long lds64(uint32_t a) {
 // Log-sum-exp merge of one unit's split partials by the 128 consumer threads
 // ("attention kernels", "prefill and decode attention"): with lse_c in the
 // log2 domain, M = max_c lse_c, w_c = 2^(lse_c - M), out = sum w_c o_c / sum w_c.
-// Each thread owns one query head and a strided set of float4 columns; the
-// weights are formed once per head and the partial rows are read four pieces
-// at a time so that the L2 round trips overlap.
+// Each thread owns one query row and a strided set of float4 columns (in two
+// passes when a unit has 32 rows); the weights are formed once per row and
+// pass, and the partial rows are read several pieces at a time so that the L2
+// round trips overlap.
 template <int D>
 __device__ __forceinline__ void merge_unit(const DecodeParams &p, long long ua, long long U,
                                            long long G, long long c_first, long long c_last,
                                            int s, int h) {
     constexpr int V4 = D / 4;                      // float4 columns per row
-    constexpr int MAXC = (V4 + 7) / 8;             // columns per thread when rows = 16
+    constexpr int MAXC = (V4 + 7) / 8;             // columns per thread and pass
     const int R = p.rows, g = p.group;
-    const int tph = kConsumers / R;                // threads per query row (R <= 16)
+    const int tph = kConsumers / R;                // threads per query row (R <= 32)
     const int head = threadIdx.x / tph, sub = threadIdx.x % tph;   // head: the query row
     if (head >= R) return;                         // 128 / R need not be exact
     // output row of query row `head`: query token head / g, head h*g + head % g
@@ -348,63 +363,71 @@ __device__ __forceinline__ void merge_unit(const DecodeParams &p, long long ua, 
     // whenever M grows (the online softmax merge).
     constexpr int NG = D == 128 ? 4 : 2;
     float M = -INFINITY, W = 0.f;
-    float4 acc[MAXC];
+    for (int cb = 0; cb < V4; cb += MAXC * tph) {
+        M = -INFINITY;
+        W = 0.f;
+        float4 acc[MAXC];
 #pragma unroll
-    for (int i = 0; i < MAXC; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (long long c = c_first; c <= c_last; c += NG) {
-        float l[NG];
-        float4 v[NG][MAXC];
+        for (int i = 0; i < MAXC; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (long long c = c_first; c <= c_last; c += NG) {
+            float l[NG];
+            float4 v[NG][MAXC];
 #pragma unroll
-        for (int k = 0; k < NG; ++k) {
-            const bool live = c + k <= c_last;
-            const long long sl = slot_of(live ? c + k : c);
-            l[k] = live ? __ldcg(p.lse_part + sl * R + head) : -INFINITY;
-            const float4 *row = reinterpret_cast<const float4 *>(p.o_part + (sl * R + head) * D);
+            for (int k = 0; k < NG; ++k) {
+                const bool live = c + k <= c_last;
+                const long long sl = slot_of(live ? c + k : c);
+                l[k] = live ? __ldcg(p.lse_part + sl * R + head) : -INFINITY;
+                const float4 *row =
+                    reinterpret_cast<const float4 *>(p.o_part + (sl * R + head) * D);
+#pragma unroll
+                for (int i = 0; i < MAXC; ++i) {
+                    const int col = cb + sub + i * tph;
+                    v[k][i] = (live && col < V4) ? __ldcg(row + col)
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+            float gm = M;
+#pragma unroll
+            for (int k = 0; k < NG; ++k) gm = fmaxf(gm, l[k]);
+            const float Mu = gm == -INFINITY ? 0.f : gm;
+            const float so = ex2(M - Mu);
+            W *= so;
 #pragma unroll
             for (int i = 0; i < MAXC; ++i) {
-                const int col = sub + i * tph;
-                v[k][i] = (live && col < V4) ? __ldcg(row + col) : make_float4(0.f, 0.f, 0.f, 0.f);
+                acc[i].x *= so; acc[i].y *= so; acc[i].z *= so; acc[i].w *= so;
             }
-        }
-        float gm = M;
 #pragma unroll
-        for (int k = 0; k < NG; ++k) gm = fmaxf(gm, l[k]);
-        const float Mu = gm == -INFINITY ? 0.f : gm;
-        const float so = ex2(M - Mu);
-        W *= so;
+            for (int k = 0; k < NG; ++k) {
+                const float w = ex2(l[k] - Mu);
+                W += w;
+#pragma unroll
+                for (int i = 0; i < MAXC; ++i) {
+                    acc[i].x += w * v[k][i].x; acc[i].y += w * v[k][i].y;
+                    acc[i].z += w * v[k][i].z; acc[i].w += w * v[k][i].w;
+                }
+            }
+            M = gm;
+        }
+        const float inv = W > 0.f ? 1.f / W : 0.f;
 #pragma unroll
         for (int i = 0; i < MAXC; ++i) {
-            acc[i].x *= so; acc[i].y *= so; acc[i].z *= so; acc[i].w *= so;
-        }
-#pragma unroll
-        for (int k = 0; k < NG; ++k) {
-            const float w = ex2(l[k] - Mu);
-            W += w;
-#pragma unroll
-            for (int i = 0; i < MAXC; ++i) {
-                acc[i].x += w * v[k][i].x; acc[i].y += w * v[k][i].y;
-                acc[i].z += w * v[k][i].z; acc[i].w += w * v[k][i].w;
-            }
-        }
-        M = gm;
-    }
-    const float inv = W > 0.f ? 1.f / W : 0.f;
-#pragma unroll
-    for (int i = 0; i < MAXC; ++i) {
-        const int col = sub + i * tph;
-        if (col < V4) {
-            if (p.out_f32) {
-                const float4 v =
-                    make_float4(acc[i].x * inv, acc[i].y * inv, acc[i].z * inv, acc[i].w * inv);
-                *reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + orow * D + 4 * col) = v;
-            } else {
-                uint2 packed;
-                packed.x = pack_bf16x2(acc[i].x * inv, acc[i].y * inv);
-                packed.y = pack_bf16x2(acc[i].z * inv, acc[i].w * inv);
-                *reinterpret_cast<uint2 *>(p.out + orow * D + 4 * col) = packed;
+            const int col = cb + sub + i * tph;
+            if (col < V4) {
+                if (p.out_f32) {
+                    const float4 v = make_float4(acc[i].x * inv, acc[i].y * inv, acc[i].z * inv,
+                                                 acc[i].w * inv);
+                    *reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + orow * D +
+                                                4 * col) = v;
+                } else {
+                    uint2 packed;
+                    packed.x = pack_bf16x2(acc[i].x * inv, acc[i].y * inv);
+                    packed.y = pack_bf16x2(acc[i].z * inv, acc[i].w * inv);
+                    *reinterpret_cast<uint2 *>(p.out + orow * D + 4 * col) = packed;
+                }
             }
         }
     }
+    // every pass saw the same weights, so M and W are those of any pass
     if (p.lse_out && sub == 0)
         p.lse_out[orow] = W > 0.f ? (M + log2f(W)) * kLn2 : -INFINITY;
 }
@@ -586,7 +609,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 const uint32_t as = ait % kAppSlots;
                 bool ok = true;
                 if (lane == 0 && ait >= (uint32_t)kAppSlots)
-                    ok = mbar_wait_bounded(app_free + 8 * as, ((ait / kAppSlots) - 1) & 1);
+                    ok = mbar_wait_bounded(app_free + 8 * as, ((ait / kAppSlots) - 1) & 1, p.wait_ns);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) {
                     if (lane == 0) raise_flag(p.flags, kFlagTimeout);
@@ -677,7 +700,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             {
                 const uint32_t slot = sit % C::NSEG;
                 if (lane == 0 && sit >= (uint32_t)C::NSEG)
-                    ok = mbar_wait_bounded(seg_empty + 8 * slot, ((sit / C::NSEG) - 1) & 1);
+                    ok = mbar_wait_bounded(seg_empty + 8 * slot, ((sit / C::NSEG) - 1) & 1, p.wait_ns);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 if (lane == 0) {
@@ -730,11 +753,11 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     const int nb = min(C::BPS, j1 - jj);
                     const uint32_t slot = it % NSTAGES;
                     if (lane == 0 && it >= (uint32_t)NSTAGES)
-                        ok = mbar_wait_bounded(bar_empty + 8 * slot, ((it / NSTAGES) - 1) & 1);
+                        ok = mbar_wait_bounded(bar_empty + 8 * slot, ((it / NSTAGES) - 1) & 1, p.wait_ns);
                     if (app_seg && jj + nb == j1 && lane == 0 && ok) {
                         // the appended row is in this stage: wait for its write
                         const uint32_t as = ait % kAppSlots;
-                        ok = mbar_wait_bounded(app_done + 8 * as, (ait / kAppSlots) & 1);
+                        ok = mbar_wait_bounded(app_done + 8 * as, (ait / kAppSlots) & 1, p.wait_ns);
                         mbar_arrive(app_free + 8 * as);
                         ++ait;
                     }
@@ -769,7 +792,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             const uint32_t slot = sit % C::NSEG;
             bool free_slot = true;
             if (sit >= (uint32_t)C::NSEG)
-                free_slot = mbar_wait_bounded(seg_empty + 8 * slot, ((sit / C::NSEG) - 1) & 1);
+                free_slot = mbar_wait_bounded(seg_empty + 8 * slot, ((sit / C::NSEG) - 1) & 1,
+                                              p.wait_ns);
             // drain: every issued copy must land before the CTA may exit.  Each
             // slot waited on here has no later arrival, so its parity is exact;
             // segment sit - NSEG is skipped once the consumers released its
@@ -777,13 +801,13 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             const uint32_t first = it > NSTAGES ? it - NSTAGES : 0;
             for (uint32_t k = first; k < it; ++k)
                 if (!mbar_wait_bounded(bar_full + 8 * (k % NSTAGES), (k / NSTAGES) & 1,
-                                       200000000ull))
+                                       kDrainWaitNs))
                     raise_flag(p.flags, kFlagTimeout);
             uint32_t qfirst = sit > C::NSEG ? sit - C::NSEG : 0;
             if (free_slot && sit >= (uint32_t)C::NSEG) qfirst = sit - C::NSEG + 1;
             for (uint32_t k = qfirst; k < sit; ++k)
                 if (!mbar_wait_bounded(seg_full + 8 * (k % C::NSEG), (k / C::NSEG) & 1,
-                                       200000000ull))
+                                       kDrainWaitNs))
                     raise_flag(p.flags, kFlagTimeout);
             // terminal descriptor (also after a timeout, so that the consumers stop)
             if (free_slot) {
@@ -801,7 +825,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
     for (;;) {
         // ---- next segment: descriptor + query fragments from shared memory
         const uint32_t qs = sit % C::NSEG;
-        const bool seg_ok = mbar_wait_bounded(seg_full + 8 * qs, (sit / C::NSEG) & 1);
+        const bool seg_ok = mbar_wait_bounded(seg_full + 8 * qs, (sit / C::NSEG) & 1, p.wait_ns);
         if (!seg_ok) raise_flag(p.flags, kFlagTimeout);
         const uint32_t da = sSeg + qs * (uint32_t)sizeof(SegDesc);
         const long long useg = lds64(da + offsetof(SegDesc, u));
@@ -819,7 +843,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         const bool whole = (j0 == jlo && j1 == nunit);
         const int R = p.rows;
 
-        const float sl2 = p.scale_log2 * ksc;
+        float sl2 = p.scale_log2 * ksc;
         // output row of query row r: query token r / g, head h*g + r % g
         auto orow = [&](int r) -> long long {
             return ((long long)s * p.q_len + r / g) * p.num_q_heads + (long long)h * g + r % g;
@@ -827,23 +851,28 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         // partial results: slot 2c for the CTA's first segment, 2c+1 for its last
         const long long pslot = 2 * cta + (useg == u0 ? 0 : 1);
         constexpr int CPR = D / 8;   // 8-float chunks per row
-        // (A + B) / L for the rows of round nt (rows 8*nt .. 8*nt + 7), 8
-        // consecutive dims per step: the output, or this CTA's partial result
-        auto finalize_rows = [&](int nt) {
+        // (A + B) / L (two merge buffers) or A / L (one) for rows r0 .. r0 + 7,
+        // 8 consecutive dims per step: the output, or this CTA's partial result
+        auto finalize_rows = [&](int r0) {
             for (int c = tid; c < 8 * CPR; c += kConsumers) {
-                const int rl = c / CPR, d0 = (c % CPR) * 8, r = nt * 8 + rl;
+                const int rl = c / CPR, d0 = (c % CPR) * 8, r = r0 + rl;
                 if (r >= R) continue;
                 const uint32_t a = sO + (rl * C::OROW + d0) * 4;
                 uint32_t x[8], y[8];
                 lds128(a, x[0], x[1], x[2], x[3]);
                 lds128(a + 16, x[4], x[5], x[6], x[7]);
-                lds128(a + C::OBUF, y[0], y[1], y[2], y[3]);
-                lds128(a + C::OBUF + 16, y[4], y[5], y[6], y[7]);
+                if constexpr (C::NOBUF == 2) {
+                    lds128(a + C::OBUF, y[0], y[1], y[2], y[3]);
+                    lds128(a + C::OBUF + 16, y[4], y[5], y[6], y[7]);
+                }
                 const float inv = rowinv[r];
                 float v[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    v[i] = (__uint_as_float(x[i]) + __uint_as_float(y[i])) * inv;
+                for (int i = 0; i < 8; ++i) {
+                    v[i] = __uint_as_float(x[i]);
+                    if constexpr (C::NOBUF == 2) v[i] += __uint_as_float(y[i]);
+                    v[i] *= inv;
+                }
                 if (whole) {
                     const long long at = orow(r) * D + d0;
                     if (p.out_f32) {
@@ -869,14 +898,20 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         };
 
         if constexpr (CC == 0) {
+            // This warp's row group: rows rbase .. rbase + 8 * NTW - 1 (all rows
+            // unless the unit has 32, when warps 0, 1 take rows 0-15 and warps 2,
+            // 3 rows 16-31)
+            const int rg = warp / C::GW;
+            const int rbase = 16 * rg;
             // visible token range [lo, hi) of the two query rows this lane holds
-            // per n-tile (rows 8*nt + 2*t4 + {0, 1}; row = query token * g + head)
-            int vis_lo[NT][2], vis_hi[NT][2];
+            // per n-tile (rows rbase + 8*nt + 2*t4 + {0, 1}; row = query token * g
+            // + head)
+            int vis_lo[C::NTW][2], vis_hi[C::NTW][2];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+            for (int nt = 0; nt < C::NTW; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const int row = nt * 8 + 2 * t4 + e;
+                    const int row = rbase + nt * 8 + 2 * t4 + e;
                     const int hi = ctx - p.q_len + 1 + row / g;
                     vis_hi[nt][e] = row < R ? hi : 0;
                     vis_lo[nt][e] = (row < R && p.window > 0) ? max(0, hi - p.window) : 0;
@@ -885,12 +920,12 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             // query fragments (B operand, Q^T[d][row]) from the slot: into
             // registers now, or (head_dim 256) by ldmatrix at every k-step
             const uint32_t qbase = sQ + qs * C::QSLOT;
-            uint32_t qf[C::QSMEM ? 1 : C::KSTEPS][NT][2];
+            uint32_t qf[C::QSMEM ? 1 : C::KSTEPS][C::NTW][2];
             if constexpr (!C::QSMEM) {
                 const uint32_t qb = qbase;
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const int head = nt * 8 + gid;      // query row held as B column
+                for (int nt = 0; nt < C::NTW; ++nt) {
+                    const int head = rbase + nt * 8 + gid;   // query row held as B column
                     const bool live = head < R;
                     const uint32_t qr = qb + (live ? head : 0) * D * 2;
 #pragma unroll
@@ -900,12 +935,46 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                             b0 = lds32(qr + (16 * k + 2 * t4) * 2);
                             b1 = lds32(qr + (16 * k + 8 + 2 * t4) * 2);
                         } else {      // k index permuted to d = 16k + 4t + {0,1 | 2,3}
-                            b0 = bf16x2_to_f16x2(lds32(qr + (16 * k + 4 * t4) * 2));
-                            b1 = bf16x2_to_f16x2(lds32(qr + (16 * k + 4 * t4 + 2) * 2));
+                            b0 = lds32(qr + (16 * k + 4 * t4) * 2);       // bf16 pairs,
+                            b1 = lds32(qr + (16 * k + 4 * t4 + 2) * 2);   // converted below
                         }
                         qf[k][nt][0] = live ? b0 : 0u;
                         qf[k][nt][1] = live ? b1 : 0u;
                     }
+                }
+                if constexpr (FP8) {
+                    // The FP8 product runs in f16, whose range is narrower than
+                    // bf16's.  The unit's query rows are scaled by a power of two
+                    // 2^sh that puts their largest magnitude in [2^14, 2^15), so no
+                    // value overflows and small ones keep their bits, and the
+                    // score scale takes 2^-sh back (both exact).  The warps of a
+                    // row group read the same rows, so they pick the same sh.
+                    float qmax = 0.f;
+#pragma unroll
+                    for (int k = 0; k < C::KSTEPS; ++k)
+#pragma unroll
+                        for (int nt = 0; nt < C::NTW; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const float2 f = unpack_bf16x2(qf[k][nt][e]);
+                                qmax = fmaxf(qmax, fmaxf(fabsf(f.x), fabsf(f.y)));
+                            }
+#pragma unroll
+                    for (int off = 16; off; off >>= 1)
+                        qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, off));
+                    const int ex = qmax > 0.f ? (int)((__float_as_uint(qmax) >> 23) & 0xffu) - 127 : 14;
+                    const int sh = min(100, max(-100, 14 - ex));
+                    const float up = __uint_as_float((uint32_t)(127 + sh) << 23);
+                    sl2 *= __uint_as_float((uint32_t)(127 - sh) << 23);
+#pragma unroll
+                    for (int k = 0; k < C::KSTEPS; ++k)
+#pragma unroll
+                        for (int nt = 0; nt < C::NTW; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const float2 f = unpack_bf16x2(qf[k][nt][e]);
+                                qf[k][nt][e] = pack_f16x2(f.x * up, f.y * up);
+                            }
                 }
             }
             if (!C::QSMEM) {
@@ -914,14 +983,15 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             }
             ++sit;
 
-            // This warp's online-softmax state over its own 16 tokens of every
-            // stage: running max and (lane-partial) sum per query row, and
-            // O^T[d][row] for all D dims.  The 4 warps' states are merged once,
-            // at the end of the segment.
-            float m_run[NT][2], l_run[NT][2];
-            float o[C::DT][NT][4];
+            // This warp's online-softmax state over its own tokens of every
+            // stage (16, or 32 with two row groups): running max and
+            // (lane-partial) sum per query row, and O^T[d][row] for all D dims.
+            // The states of a row group's warps are merged once, at the end of
+            // the segment.
+            float m_run[C::NTW][2], l_run[C::NTW][2];
+            float o[C::DT][C::NTW][4];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
+            for (int nt = 0; nt < C::NTW; ++nt) {
                 m_run[nt][0] = m_run[nt][1] = -INFINITY;
                 l_run[nt][0] = l_run[nt][1] = 0.f;
 #pragma unroll
@@ -937,7 +1007,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 // segment or with the context)
                 const int n_valid = min(ctx - jj * BS, nb * BS);
                 const uint32_t slot = it % NSTAGES;
-                const bool ok = mbar_wait_bounded(bar_full + 8 * slot, (it / NSTAGES) & 1);
+                const bool ok = mbar_wait_bounded(bar_full + 8 * slot, (it / NSTAGES) & 1, p.wait_ns);
                 ++it;
                 if (!ok) {
                     raise_flag(p.flags, kFlagTimeout);
@@ -946,221 +1016,225 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 }
                 const uint32_t sK = sbase + slot * C::STAGE, sV = sK + C::STAGE_KV;
 
-                if (16 * warp < n_valid) {
-                    // ---- S^T = K . Q^T for this warp's 16 tokens (two MMA chains)
-                    float sacc[NT][4], sac2[NT][4];
+                for (int sub = 0; sub < C::SUBS; ++sub) {
+                    // first stage token of this warp's 16-token sub-tile
+                    const int tb = C::RG == 1 ? 16 * warp : 32 * (warp & 1) + 16 * sub;
+                    if (tb < n_valid) {
+                        // ---- S^T = K . Q^T for this warp's 16 tokens (two MMA chains)
+                        float sacc[C::NTW][4], sac2[C::NTW][4];
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
+                        for (int nt = 0; nt < C::NTW; ++nt)
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) sacc[nt][e] = sac2[nt][e] = 0.f;
-                    if (!FP8) {
-                        const int mi = lane >> 3;
-                        const int tok = 16 * warp + (mi & 1) * 8 + (lane & 7);
-                        const int row = tok % BS;
-                        const uint32_t rowaddr = sK + (tok / BS) * C::TILE + row * 128;
-                        uint32_t qb4[NT][4];   // shared-memory query fragments of k, k + 1
-#pragma unroll
-                        for (int k = 0; k < C::KSTEPS; ++k) {
-                            const int chunk = 2 * k + (mi >> 1);
-                            const uint32_t addr = rowaddr + (chunk >> 3) * (BS * 128) +
-                                                  (((chunk & 7) ^ (row & 7)) << 4);
-                            uint32_t a0, a1, a2, a3;
-                            ldsm_x4(addr, a0, a1, a2, a3);
-                            if constexpr (C::QSMEM) {
-                                if ((k & 1) == 0) {
-                                    // matrices: rows nt*8 .. +7 at d = 16k, 16k+8, 16k+16, 16k+24
-#pragma unroll
-                                    for (int nt = 0; nt < NT; ++nt)
-                                        ldsm_x4(qbase + (nt * 8 + (lane & 7)) * C::QROW +
-                                                    (16 * (k + (lane >> 4)) + 8 * ((lane >> 3) & 1)) * 2,
-                                                qb4[nt][0], qb4[nt][1], qb4[nt][2], qb4[nt][3]);
-                                }
-                            }
-#pragma unroll
-                            for (int nt = 0; nt < NT; ++nt) {
-                                uint32_t b0, b1;
-                                if constexpr (C::QSMEM) {
-                                    b0 = qb4[nt][(k & 1) * 2];
-                                    b1 = qb4[nt][(k & 1) * 2 + 1];
-                                } else {
-                                    b0 = qf[k][nt][0];
-                                    b1 = qf[k][nt][1];
-                                }
-                                if (k & 1) mma_bf16(sac2[nt], a0, a1, a2, a3, b0, b1);
-                                else       mma_bf16(sacc[nt], a0, a1, a2, a3, b0, b1);
-                            }
-                        }
-                    } else {
-                        const int tok0 = 16 * warp + gid, tok1 = tok0 + 8;
-                        const int r0 = tok0 % BS, r1 = tok1 % BS;
-                        const uint32_t base0 = sK + (tok0 / BS) * C::TILE + r0 * 128 + 4 * t4;
-                        const uint32_t base1 = sK + (tok1 / BS) * C::TILE + r1 * 128 + 4 * t4;
-#pragma unroll
-                        for (int k = 0; k < C::KSTEPS; ++k) {
-                            const uint32_t w0 = lds32(base0 + ((k ^ (r0 & 7)) << 4));
-                            const uint32_t w1 = lds32(base1 + ((k ^ (r1 & 7)) << 4));
-                            const uint32_t a0 = e4m3x2_to_f16x2(w0 & 0xffffu);
-                            const uint32_t a2 = e4m3x2_to_f16x2(w0 >> 16);
-                            const uint32_t a1 = e4m3x2_to_f16x2(w1 & 0xffffu);
-                            const uint32_t a3 = e4m3x2_to_f16x2(w1 >> 16);
-#pragma unroll
-                            for (int nt = 0; nt < NT; ++nt) {
-                                if (k & 1) mma_f16(sac2[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
-                                else       mma_f16(sacc[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
-                            }
-                        }
-                    }
-
-                    // ---- mask, this warp's max per row, weights p ----------------
-                    float mx[NT][2], alpha[NT][2];
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            // stage token (only the first n_valid were loaded) and
-                            // its absolute position; the row's visible range
-                            // excludes padding rows and positions past ctx
-                            const int tok = 16 * warp + gid + (e >> 1) * 8;
-                            const int pos = jj * BS + tok;
-                            const float v = sacc[nt][e] + sac2[nt][e];
-                            sacc[nt][e] = (tok < n_valid && pos >= vis_lo[nt][e & 1] &&
-                                           pos < vis_hi[nt][e & 1])
-                                              ? v * sl2 : -INFINITY;
-                        }
-                        mx[nt][0] = fmaxf(sacc[nt][0], sacc[nt][2]);
-                        mx[nt][1] = fmaxf(sacc[nt][1], sacc[nt][3]);
-#pragma unroll
-                        for (int off = 4; off < 32; off <<= 1) {
-                            mx[nt][0] = fmaxf(mx[nt][0], __shfl_xor_sync(0xffffffffu, mx[nt][0], off));
-                            mx[nt][1] = fmaxf(mx[nt][1], __shfl_xor_sync(0xffffffffu, mx[nt][1], off));
-                        }
-                    }
-                    // Lazy rescaling: a row keeps its reference max m_run (the
-                    // exponent offset of every weight it has summed) until a
-                    // score exceeds it by more than 2^8, so weights stay below
-                    // 256 and the accumulator is rescaled only in the stages
-                    // where some row of the warp moves.
-                    bool moved = false;
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                        for (int e = 0; e < 2; ++e)
-                            moved |= mx[nt][e] > m_run[nt][e] + kLazyRescale;
-                    const bool any_moved = __any_sync(0xffffffffu, moved);
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            alpha[nt][e] = 1.f;
-                            if (any_moved && mx[nt][e] > m_run[nt][e] + kLazyRescale) {
-                                alpha[nt][e] = ex2(m_run[nt][e] - mx[nt][e]);
-                                m_run[nt][e] = mx[nt][e];
-                            }
-                            mx[nt][e] = m_run[nt][e] == -INFINITY ? 0.f : m_run[nt][e];
-                        }
-                    // rows past the end of the context may hold anything (NaN,
-                    // Inf): zero this warp's invalid V rows so that 0 * V stays 0
-                    if (n_valid < 16 * warp + 16) {
-                        const int first = max(16 * warp, n_valid), last = 16 * warp + 16;
-                        const int lines = (last - first) * C::LINES;
-                        for (int i = lane >> 3; i < lines; i += 4) {
-                            const int tok = first + i / C::LINES, ln = i % C::LINES;
-                            const uint32_t a = sV + (tok / BS) * C::TILE + ln * (BS * 128) +
-                                               (tok % BS) * 128 + (lane & 7) * 16;
-                            sts128(a, 0u, 0u, 0u, 0u);
-                        }
-                        // order these generic-proxy writes before the next TMA
-                        // into the slot
-                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                        __syncwarp();
-                    }
-
-                    // ---- P^T fragments (B operand, k = token, n = row) ------------
-                    // The score accumulator holds S^T[token][row] in the fragment
-                    // layout (lane 4r + c: tokens r and r + 8, rows 2c, 2c + 1); a
-                    // warp transpose of each 8x8 half gives P^T[row][token] in
-                    // the B-operand layout of the PV product.
-                    uint32_t pb[NT][2], pl[NT][2];
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        float pr[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) pr[e] = ex2(sacc[nt][e] - mx[nt][e & 1]);
+                            for (int e = 0; e < 4; ++e) sacc[nt][e] = sac2[nt][e] = 0.f;
                         if (!FP8) {
-                            // p = hi + lo, both bf16; the normaliser sums the fp32 p
-                            const uint32_t h0 = pack_bf16x2(pr[0], pr[1]);
-                            const uint32_t h1 = pack_bf16x2(pr[2], pr[3]);
-                            const float2 q0 = unpack_bf16x2(h0), q1 = unpack_bf16x2(h1);
-                            const uint32_t l0 = pack_bf16x2(pr[0] - q0.x, pr[1] - q0.y);
-                            const uint32_t l1 = pack_bf16x2(pr[2] - q1.x, pr[3] - q1.y);
-                            l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + pr[0] + pr[2];
-                            l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + pr[1] + pr[3];
-                            pb[nt][0] = movmatrix_trans(h0);
-                            pb[nt][1] = movmatrix_trans(h1);
-                            pl[nt][0] = movmatrix_trans(l0);
-                            pl[nt][1] = movmatrix_trans(l1);
+                            const int mi = lane >> 3;
+                            const int tok = tb + (mi & 1) * 8 + (lane & 7);
+                            const int row = tok % BS;
+                            const uint32_t rowaddr = sK + (tok / BS) * C::TILE + row * 128;
+                            uint32_t qb4[C::NTW][4];   // shared-memory query fragments of k, k + 1
+#pragma unroll
+                            for (int k = 0; k < C::KSTEPS; ++k) {
+                                const int chunk = 2 * k + (mi >> 1);
+                                const uint32_t addr = rowaddr + (chunk >> 3) * (BS * 128) +
+                                                      (((chunk & 7) ^ (row & 7)) << 4);
+                                uint32_t a0, a1, a2, a3;
+                                ldsm_x4(addr, a0, a1, a2, a3);
+                                if constexpr (C::QSMEM) {
+                                    if ((k & 1) == 0) {
+                                        // matrices: rows nt*8 .. +7 at d = 16k, 16k+8, 16k+16, 16k+24
+#pragma unroll
+                                        for (int nt = 0; nt < C::NTW; ++nt)
+                                            ldsm_x4(qbase + (rbase + nt * 8 + (lane & 7)) * C::QROW +
+                                                        (16 * (k + (lane >> 4)) + 8 * ((lane >> 3) & 1)) * 2,
+                                                    qb4[nt][0], qb4[nt][1], qb4[nt][2], qb4[nt][3]);
+                                    }
+                                }
+#pragma unroll
+                                for (int nt = 0; nt < C::NTW; ++nt) {
+                                    uint32_t b0, b1;
+                                    if constexpr (C::QSMEM) {
+                                        b0 = qb4[nt][(k & 1) * 2];
+                                        b1 = qb4[nt][(k & 1) * 2 + 1];
+                                    } else {
+                                        b0 = qf[k][nt][0];
+                                        b1 = qf[k][nt][1];
+                                    }
+                                    if (k & 1) mma_bf16(sac2[nt], a0, a1, a2, a3, b0, b1);
+                                    else       mma_bf16(sacc[nt], a0, a1, a2, a3, b0, b1);
+                                }
+                            }
                         } else {
-                            // f16 weights; the normaliser sums exactly the rounded values
-                            const uint32_t h0 = pack_f16x2(pr[0], pr[1]);
-                            const uint32_t h1 = pack_f16x2(pr[2], pr[3]);
-                            const float2 q0 = unpack_f16x2(h0), q1 = unpack_f16x2(h1);
-                            l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + q0.x + q1.x;
-                            l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + q0.y + q1.y;
-                            pb[nt][0] = movmatrix_trans(h0);
-                            pb[nt][1] = movmatrix_trans(h1);
-                        }
-                    }
-
-                    // ---- O^T += V^T . P^T over all D for this warp's tokens ------
-                    if (any_moved) {
+                            const int tok0 = tb + gid, tok1 = tok0 + 8;
+                            const int r0 = tok0 % BS, r1 = tok1 % BS;
+                            const uint32_t base0 = sK + (tok0 / BS) * C::TILE + r0 * 128 + 4 * t4;
+                            const uint32_t base1 = sK + (tok1 / BS) * C::TILE + r1 * 128 + 4 * t4;
 #pragma unroll
-                        for (int mt = 0; mt < C::DT; ++mt)
+                            for (int k = 0; k < C::KSTEPS; ++k) {
+                                const uint32_t w0 = lds32(base0 + ((k ^ (r0 & 7)) << 4));
+                                const uint32_t w1 = lds32(base1 + ((k ^ (r1 & 7)) << 4));
+                                const uint32_t a0 = e4m3x2_to_f16x2(w0 & 0xffffu);
+                                const uint32_t a2 = e4m3x2_to_f16x2(w0 >> 16);
+                                const uint32_t a1 = e4m3x2_to_f16x2(w1 & 0xffffu);
+                                const uint32_t a3 = e4m3x2_to_f16x2(w1 >> 16);
 #pragma unroll
-                            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) o[mt][nt][e] *= alpha[nt][e & 1];
-                    }
-                    if (!FP8) {
-                        const int mi = lane >> 3;
-                        const int tok = 16 * warp + (mi >> 1) * 8 + (lane & 7);
-                        const int row = tok % BS;
-                        const uint32_t rowaddr = sV + (tok / BS) * C::TILE + row * 128;
-#pragma unroll
-                        for (int mt = 0; mt < C::DT; ++mt) {
-                            const int chunk = 2 * mt + (mi & 1);
-                            const uint32_t addr = rowaddr + (chunk >> 3) * (BS * 128) +
-                                                  (((chunk & 7) ^ (row & 7)) << 4);
-                            uint32_t a0, a1, a2, a3;
-                            ldsm_x4_t(addr, a0, a1, a2, a3);
-#pragma unroll
-                            for (int nt = 0; nt < NT; ++nt) {
-                                mma_bf16(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
-                                mma_bf16(o[mt][nt], a0, a1, a2, a3, pl[nt][0], pl[nt][1]);
+                                for (int nt = 0; nt < C::NTW; ++nt) {
+                                    if (k & 1) mma_f16(sac2[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
+                                    else       mma_f16(sacc[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
+                                }
                             }
                         }
-                    } else {
-                        // tokens 2c, 2c+1, 2c+8, 2c+9 of this warp; 16 bytes at
-                        // d = 16*gid .. 16*gid + 15 (m-tile mt: bytes 2mt, 2mt+1)
-                        uint32_t wv[4][4];
+
+                        // ---- mask, this warp's max per row, weights p ----------------
+                        float mx[C::NTW][2], alpha[C::NTW][2];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const int tok = 16 * warp + 2 * t4 + (q & 1) + (q >> 1) * 8;
-                            const int row = tok % BS;
-                            lds128(sV + (tok / BS) * C::TILE + row * 128 + ((gid ^ (row & 7)) << 4),
-                                   wv[q][0], wv[q][1], wv[q][2], wv[q][3]);
+                        for (int nt = 0; nt < C::NTW; ++nt) {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                // stage token (only the first n_valid were loaded) and
+                                // its absolute position; the row's visible range
+                                // excludes padding rows and positions past ctx
+                                const int tok = tb + gid + (e >> 1) * 8;
+                                const int pos = jj * BS + tok;
+                                const float v = sacc[nt][e] + sac2[nt][e];
+                                sacc[nt][e] = (tok < n_valid && pos >= vis_lo[nt][e & 1] &&
+                                               pos < vis_hi[nt][e & 1])
+                                                  ? v * sl2 : -INFINITY;
+                            }
+                            mx[nt][0] = fmaxf(sacc[nt][0], sacc[nt][2]);
+                            mx[nt][1] = fmaxf(sacc[nt][1], sacc[nt][3]);
+#pragma unroll
+                            for (int off = 4; off < 32; off <<= 1) {
+                                mx[nt][0] = fmaxf(mx[nt][0], __shfl_xor_sync(0xffffffffu, mx[nt][0], off));
+                                mx[nt][1] = fmaxf(mx[nt][1], __shfl_xor_sync(0xffffffffu, mx[nt][1], off));
+                            }
                         }
+                        // Lazy rescaling: a row keeps its reference max m_run (the
+                        // exponent offset of every weight it has summed) until a
+                        // score exceeds it by more than 2^8, so weights stay below
+                        // 256 and the accumulator is rescaled only in the stages
+                        // where some row of the warp moves.
+                        bool moved = false;
 #pragma unroll
-                        for (int mt = 0; mt < C::DT; ++mt) {
-                            const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
-                            const uint32_t x = prmt(wv[0][mt >> 1], wv[1][mt >> 1], sel);
-                            const uint32_t y = prmt(wv[2][mt >> 1], wv[3][mt >> 1], sel);
-                            const uint32_t a0 = e4m3x2_to_f16x2(x & 0xffffu);
-                            const uint32_t a1 = e4m3x2_to_f16x2(x >> 16);
-                            const uint32_t a2 = e4m3x2_to_f16x2(y & 0xffffu);
-                            const uint32_t a3 = e4m3x2_to_f16x2(y >> 16);
+                        for (int nt = 0; nt < C::NTW; ++nt)
 #pragma unroll
-                            for (int nt = 0; nt < NT; ++nt)
-                                mma_f16(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+                            for (int e = 0; e < 2; ++e)
+                                moved |= mx[nt][e] > m_run[nt][e] + kLazyRescale;
+                        const bool any_moved = __any_sync(0xffffffffu, moved);
+#pragma unroll
+                        for (int nt = 0; nt < C::NTW; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                alpha[nt][e] = 1.f;
+                                if (any_moved && mx[nt][e] > m_run[nt][e] + kLazyRescale) {
+                                    alpha[nt][e] = ex2(m_run[nt][e] - mx[nt][e]);
+                                    m_run[nt][e] = mx[nt][e];
+                                }
+                                mx[nt][e] = m_run[nt][e] == -INFINITY ? 0.f : m_run[nt][e];
+                            }
+                        // rows past the end of the context may hold anything (NaN,
+                        // Inf): zero this warp's invalid V rows so that 0 * V stays 0
+                        if (n_valid < tb + 16) {
+                            const int first = max(tb, n_valid), last = tb + 16;
+                            const int lines = (last - first) * C::LINES;
+                            for (int i = lane >> 3; i < lines; i += 4) {
+                                const int tok = first + i / C::LINES, ln = i % C::LINES;
+                                const uint32_t a = sV + (tok / BS) * C::TILE + ln * (BS * 128) +
+                                                   (tok % BS) * 128 + (lane & 7) * 16;
+                                sts128(a, 0u, 0u, 0u, 0u);
+                            }
+                            // order these generic-proxy writes before the next TMA
+                            // into the slot
+                            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                            __syncwarp();
+                        }
+
+                        // ---- P^T fragments (B operand, k = token, n = row) ------------
+                        // The score accumulator holds S^T[token][row] in the fragment
+                        // layout (lane 4r + c: tokens r and r + 8, rows 2c, 2c + 1); a
+                        // warp transpose of each 8x8 half gives P^T[row][token] in
+                        // the B-operand layout of the PV product.
+                        uint32_t pb[C::NTW][2], pl[C::NTW][2];
+#pragma unroll
+                        for (int nt = 0; nt < C::NTW; ++nt) {
+                            float pr[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) pr[e] = ex2(sacc[nt][e] - mx[nt][e & 1]);
+                            if (!FP8) {
+                                // p = hi + lo, both bf16; the normaliser sums the fp32 p
+                                const uint32_t h0 = pack_bf16x2(pr[0], pr[1]);
+                                const uint32_t h1 = pack_bf16x2(pr[2], pr[3]);
+                                const float2 q0 = unpack_bf16x2(h0), q1 = unpack_bf16x2(h1);
+                                const uint32_t l0 = pack_bf16x2(pr[0] - q0.x, pr[1] - q0.y);
+                                const uint32_t l1 = pack_bf16x2(pr[2] - q1.x, pr[3] - q1.y);
+                                l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + pr[0] + pr[2];
+                                l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + pr[1] + pr[3];
+                                pb[nt][0] = movmatrix_trans(h0);
+                                pb[nt][1] = movmatrix_trans(h1);
+                                pl[nt][0] = movmatrix_trans(l0);
+                                pl[nt][1] = movmatrix_trans(l1);
+                            } else {
+                                // f16 weights; the normaliser sums exactly the rounded values
+                                const uint32_t h0 = pack_f16x2(pr[0], pr[1]);
+                                const uint32_t h1 = pack_f16x2(pr[2], pr[3]);
+                                const float2 q0 = unpack_f16x2(h0), q1 = unpack_f16x2(h1);
+                                l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + q0.x + q1.x;
+                                l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + q0.y + q1.y;
+                                pb[nt][0] = movmatrix_trans(h0);
+                                pb[nt][1] = movmatrix_trans(h1);
+                            }
+                        }
+
+                        // ---- O^T += V^T . P^T over all D for this warp's tokens ------
+                        if (any_moved) {
+#pragma unroll
+                            for (int mt = 0; mt < C::DT; ++mt)
+#pragma unroll
+                                for (int nt = 0; nt < C::NTW; ++nt)
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) o[mt][nt][e] *= alpha[nt][e & 1];
+                        }
+                        if (!FP8) {
+                            const int mi = lane >> 3;
+                            const int tok = tb + (mi >> 1) * 8 + (lane & 7);
+                            const int row = tok % BS;
+                            const uint32_t rowaddr = sV + (tok / BS) * C::TILE + row * 128;
+#pragma unroll
+                            for (int mt = 0; mt < C::DT; ++mt) {
+                                const int chunk = 2 * mt + (mi & 1);
+                                const uint32_t addr = rowaddr + (chunk >> 3) * (BS * 128) +
+                                                      (((chunk & 7) ^ (row & 7)) << 4);
+                                uint32_t a0, a1, a2, a3;
+                                ldsm_x4_t(addr, a0, a1, a2, a3);
+#pragma unroll
+                                for (int nt = 0; nt < C::NTW; ++nt) {
+                                    mma_bf16(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+                                    mma_bf16(o[mt][nt], a0, a1, a2, a3, pl[nt][0], pl[nt][1]);
+                                }
+                            }
+                        } else {
+                            // tokens 2c, 2c+1, 2c+8, 2c+9 of this warp; 16 bytes at
+                            // d = 16*gid .. 16*gid + 15 (m-tile mt: bytes 2mt, 2mt+1)
+                            uint32_t wv[4][4];
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const int tok = tb + 2 * t4 + (q & 1) + (q >> 1) * 8;
+                                const int row = tok % BS;
+                                lds128(sV + (tok / BS) * C::TILE + row * 128 + ((gid ^ (row & 7)) << 4),
+                                       wv[q][0], wv[q][1], wv[q][2], wv[q][3]);
+                            }
+#pragma unroll
+                            for (int mt = 0; mt < C::DT; ++mt) {
+                                const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+                                const uint32_t x = prmt(wv[0][mt >> 1], wv[1][mt >> 1], sel);
+                                const uint32_t y = prmt(wv[2][mt >> 1], wv[3][mt >> 1], sel);
+                                const uint32_t a0 = e4m3x2_to_f16x2(x & 0xffffu);
+                                const uint32_t a1 = e4m3x2_to_f16x2(x >> 16);
+                                const uint32_t a2 = e4m3x2_to_f16x2(y & 0xffffu);
+                                const uint32_t a3 = e4m3x2_to_f16x2(y >> 16);
+#pragma unroll
+                                for (int nt = 0; nt < C::NTW; ++nt)
+                                    mma_f16(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+                            }
                         }
                     }
                 }
@@ -1172,10 +1246,12 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 if (lane == 0) mbar_arrive(seg_empty + 8 * qs);   // query rows read
             }
 
-            // ---- finish the segment: merge the 4 warps' states -----------------
-            // In a fixed order, so that results do not depend on timing: warps 1
-            // and 3 store their O rows (buffers A and B), warps 0 and 2 add theirs
-            // to them with both weights, and the output is (A + B) / L.
+            // ---- finish the segment: merge the warps' states -------------------
+            // In a fixed order, so that results do not depend on timing.  With one
+            // row group, warps 1 and 3 store their O rows (buffers A and B), warps
+            // 0 and 2 add theirs to them with both weights, and the output is
+            // (A + B) / L.  With two row groups (32 rows), each group's odd warp
+            // stores, its even warp adds, and the output is that buffer / L.
             // output dim held by accumulator element (mt, e)
             auto dim_of = [&](int mt, int e) -> int {
                 if (!FP8) return 16 * mt + gid + (e >> 1) * 8;
@@ -1183,62 +1259,70 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             };
             // A: warps 0, 1; B: warps 2, 3
             auto store_rows = [&](int nt) {
-                float *buf = reinterpret_cast<float *>(smem + C::OFF_O + (warp >> 1) * C::OBUF);
+                float *buf = reinterpret_cast<float *>(
+                    smem + C::OFF_O + (C::NOBUF == 2 ? (warp >> 1) : 0) * C::OBUF);
 #pragma unroll
                 for (int mt = 0; mt < C::DT; ++mt)
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         buf[(2 * t4 + (e & 1)) * C::OROW + dim_of(mt, e)] = o[mt][nt][e];
             };
-            if (warp & 1) store_rows(0);
+            if ((warp & 1) && rg == 0) store_rows(0);
             // row sums over this warp's lanes; row max and sum of every warp
             // through shared memory; all consumers agree on leaving after a timeout
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+            for (int nt = 0; nt < C::NTW; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     float v = l_run[nt][e];
 #pragma unroll
                     for (int off = 4; off < 32; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
                     if (gid == 0) {
-                        red[warp * C::NP + nt * 8 + 2 * t4 + e] = m_run[nt][e];
-                        lsum[warp * C::NP + nt * 8 + 2 * t4 + e] = v;
+                        red[warp * C::NP + rbase + nt * 8 + 2 * t4 + e] = m_run[nt][e];
+                        lsum[warp * C::NP + rbase + nt * 8 + 2 * t4 + e] = v;
                     }
                 }
             if (named_bar_sync_or(kBarConsumers, kConsumers, abort)) return;
-            // weights of this warp's and its partner's (warp + 1) O in the merged row
-            float wsc[NT][2], psc[NT][2];
+            // weights of this warp's and its partner's (warp + 1) O in the merged
+            // row; the row's max and sum run over the warps of its row group
+            const int w0 = rg * C::GW;
+            float wsc[C::NTW][2], psc[C::NTW][2];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+            for (int nt = 0; nt < C::NTW; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const int r = nt * 8 + 2 * t4 + e;
+                    const int r = rbase + nt * 8 + 2 * t4 + e;
                     float M = -INFINITY;
 #pragma unroll
-                    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[w * C::NP + r]);
+                    for (int w = 0; w < C::GW; ++w) M = fmaxf(M, red[(w0 + w) * C::NP + r]);
                     const float Mu = M == -INFINITY ? 0.f : M;
                     wsc[nt][e] = ex2(m_run[nt][e] - Mu);
                     psc[nt][e] = ex2(red[((warp + 1) & 3) * C::NP + r] - Mu);
-                    if (warp == 0 && gid == 0) {
+                    if (warp == w0 && gid == 0) {
                         float L = 0.f;
 #pragma unroll
-                        for (int w = 0; w < kConsumerWarps; ++w)
-                            L += lsum[w * C::NP + r] * ex2(red[w * C::NP + r] - Mu);
+                        for (int w = 0; w < C::GW; ++w)
+                            L += lsum[(w0 + w) * C::NP + r] * ex2(red[(w0 + w) * C::NP + r] - Mu);
                         rowinv[r] = L > 0.f ? vsc / L : 0.f;
                         rowlse[r] = L > 0.f ? M + log2f(L) : -INFINITY;
                     }
                 }
 
+            // Rounds of 8 rows: with two buffers both halves of the warps merge
+            // rows 8*nt .. 8*nt + 7 together (A: warps 0, 1; B: warps 2, 3); with
+            // two row groups one buffer serves the group of the round.
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                if (nt > 0) {
-                    named_bar_sync(kBarConsumers, kConsumers);   // A and B read
-                    if (warp & 1) store_rows(nt);
+            for (int rd = 0; rd < C::RG * C::NTW; ++rd) {
+                const int grp = rd / C::NTW, nt = rd % C::NTW;
+                if (rd > 0) {
+                    named_bar_sync(kBarConsumers, kConsumers);   // buffers read
+                    if ((warp & 1) && rg == grp) store_rows(nt);
                     named_bar_sync(kBarConsumers, kConsumers);
                 }
-                // warps 0 and 2: buffer = own O * weight + partner's O * its weight
-                if (!(warp & 1)) {
-                    float *buf = reinterpret_cast<float *>(smem + C::OFF_O + (warp >> 1) * C::OBUF);
+                // even warps: buffer = own O * weight + partner's O * its weight
+                if (!(warp & 1) && rg == grp) {
+                    float *buf = reinterpret_cast<float *>(
+                        smem + C::OFF_O + (C::NOBUF == 2 ? (warp >> 1) : 0) * C::OBUF);
                     float part[C::DT][4];
 #pragma unroll
                     for (int mt = 0; mt < C::DT; ++mt)
@@ -1253,7 +1337,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                 o[mt][nt][e] * wsc[nt][e & 1] + part[mt][e] * psc[nt][e & 1];
                 }
                 named_bar_sync(kBarConsumers, kConsumers);
-                finalize_rows(nt);
+                finalize_rows(grp * 16 + nt * 8);
             }
         } else {
             // ---- CUDA-core variant: FMA dot products, warp-shuffle sums --------
@@ -1314,7 +1398,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 const int nb = min(C::BPS, j1 - jj);
                 const int n_valid = min(ctx - jj * BS, nb * BS);
                 const uint32_t slot = it % NSTAGES;
-                const bool ok = mbar_wait_bounded(bar_full + 8 * slot, (it / NSTAGES) & 1);
+                const bool ok = mbar_wait_bounded(bar_full + 8 * slot, (it / NSTAGES) & 1, p.wait_ns);
                 ++it;
                 if (!ok) {
                     raise_flag(p.flags, kFlagTimeout);

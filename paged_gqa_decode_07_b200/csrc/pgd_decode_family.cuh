@@ -71,12 +71,18 @@ int decode_ctas_per_sm() {
     template cudaError_t launch_decode<D, 16, 2, FP8>(const DecodeLaunchArgs &); \
     template cudaError_t launch_decode<D, 32, 2, FP8>(const DecodeLaunchArgs &); \
     template cudaError_t launch_decode<D, 64, 2, FP8>(const DecodeLaunchArgs &); \
+    template cudaError_t launch_decode<D, 16, 4, FP8>(const DecodeLaunchArgs &); \
+    template cudaError_t launch_decode<D, 32, 4, FP8>(const DecodeLaunchArgs &); \
+    template cudaError_t launch_decode<D, 64, 4, FP8>(const DecodeLaunchArgs &); \
     template int decode_ctas_per_sm<D, 16, 1, FP8>();                           \
     template int decode_ctas_per_sm<D, 32, 1, FP8>();                           \
     template int decode_ctas_per_sm<D, 64, 1, FP8>();                           \
     template int decode_ctas_per_sm<D, 16, 2, FP8>();                           \
     template int decode_ctas_per_sm<D, 32, 2, FP8>();                           \
-    template int decode_ctas_per_sm<D, 64, 2, FP8>();
+    template int decode_ctas_per_sm<D, 64, 2, FP8>();                           \
+    template int decode_ctas_per_sm<D, 16, 4, FP8>();                           \
+    template int decode_ctas_per_sm<D, 32, 4, FP8>();                           \
+    template int decode_ctas_per_sm<D, 64, 4, FP8>();
 
 // CUDA-core comparison variants (bf16, head_dim 128, up to CC query rows)
 #define PGD_INSTANTIATE_CUDA_CORE(CC)                                             \

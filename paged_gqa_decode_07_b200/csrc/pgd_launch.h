@@ -39,12 +39,18 @@ int decode_ctas_per_sm();
     extern template cudaError_t launch_decode<D, 16, 2, FP8>(const DecodeLaunchArgs &); \
     extern template cudaError_t launch_decode<D, 32, 2, FP8>(const DecodeLaunchArgs &); \
     extern template cudaError_t launch_decode<D, 64, 2, FP8>(const DecodeLaunchArgs &); \
+    extern template cudaError_t launch_decode<D, 16, 4, FP8>(const DecodeLaunchArgs &); \
+    extern template cudaError_t launch_decode<D, 32, 4, FP8>(const DecodeLaunchArgs &); \
+    extern template cudaError_t launch_decode<D, 64, 4, FP8>(const DecodeLaunchArgs &); \
     extern template int decode_ctas_per_sm<D, 16, 1, FP8>();                           \
     extern template int decode_ctas_per_sm<D, 32, 1, FP8>();                           \
     extern template int decode_ctas_per_sm<D, 64, 1, FP8>();                           \
     extern template int decode_ctas_per_sm<D, 16, 2, FP8>();                           \
     extern template int decode_ctas_per_sm<D, 32, 2, FP8>();                           \
-    extern template int decode_ctas_per_sm<D, 64, 2, FP8>();
+    extern template int decode_ctas_per_sm<D, 64, 2, FP8>();                           \
+    extern template int decode_ctas_per_sm<D, 16, 4, FP8>();                           \
+    extern template int decode_ctas_per_sm<D, 32, 4, FP8>();                           \
+    extern template int decode_ctas_per_sm<D, 64, 4, FP8>();
 
 PGD_DECLARE_FAMILY(128, false)
 PGD_DECLARE_FAMILY(256, false)

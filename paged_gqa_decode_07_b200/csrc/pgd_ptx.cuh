@@ -60,12 +60,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Limits of the bounded waits.  Pipeline waits (a stage, a descriptor, an
+// appended row) give up after DecodeParams::wait_ns, 1 s unless a test
+// shortens it; the producer's final drain of its own copies always allows
+// kDrainWaitNs, because every copy it issued must land before the CTA exits.
+constexpr uint64_t kDefaultWaitNs = 1000000000ull;
+constexpr uint64_t kDrainWaitNs = 200000000ull;
+
 // Wait for the phase with the given parity to complete, for at most
 // `limit_ns` nanoseconds.  Returns false if the limit passed; the caller
 // raises the timeout flag, keeps its control flow uniform and bails out at
 // the next point where the whole CTA can agree.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  uint64_t limit_ns = 1000000000ull) {
+                                                  uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
@@ -200,13 +207,6 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t v) {
 __device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
     __half2 h = *reinterpret_cast<__half2 *>(&v);
     return __half22float2(h);
-}
-
-// bf16 pair -> f16 pair (through fp32; exact for magnitudes in f16's
-// normal range, rounded to nearest otherwise).
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
-    float2 f = unpack_bf16x2(v);
-    return pack_f16x2(f.x, f.y);
 }
 
 // Hardware base-2 exponential (ex2.approx); exp2(-inf) = 0.

@@ -19,7 +19,8 @@ OK, INVALID, UNSUPPORTED, CUDA, BOUNDS, TIMEOUT, WORKSPACE = range(7)
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return re.findall(r"^\s*(?:pgd_status|size_t|const\s+char\s*\*)\s*\**\s*(\w+)\s*\(",
+    return re.findall(r"^\s*(?:pgd_status|pgd_decode_math|size_t|uint64_t|const\s+char\s*\*)"
+                      r"\s*\**\s*(\w+)\s*\(",
                       text, flags=re.M)
 
 
@@ -122,11 +123,13 @@ def decode_ex(lib, q_len, window, **kw):
 @pytest.mark.parametrize("q_len,window,kw,status", [
     (0, 0, {}, INVALID),                   # no query token
     (1, -1, {}, INVALID),                  # negative window
-    (5, 0, {}, UNSUPPORTED),               # g * q_len = 20 rows > 16
-    (2, 0, dict(Hq=16, Hkv=1), UNSUPPORTED),
+    (9, 0, {}, UNSUPPORTED),               # g * q_len = 36 rows > 32
+    (3, 0, dict(Hq=16, Hkv=1), UNSUPPORTED),
     (4, 3, dict(out=MIS), INVALID),
     (4, 3, dict(B=0, q=None), OK),
     (8, 0, dict(Hq=4, Hkv=2, B=0), OK),    # 16 rows: accepted
+    (8, 0, dict(B=0), OK),                 # 32 rows (g 4, q_len 8): accepted
+    (2, 0, dict(Hq=16, Hkv=1, D=256, B=0), OK),   # 32 rows at head_dim 256
 ])
 def test_decode_ex_host_validation(lib, q_len, window, kw, status):
     assert decode_ex(lib, q_len, window, **kw) == status
@@ -176,3 +179,13 @@ def test_decode_math_setting_is_host_only(lib):
     assert lib.pgd_set_decode_math(1) == OK and lib.pgd_get_decode_math() == 1
     assert lib.pgd_set_decode_math(7) == INVALID and lib.pgd_get_decode_math() == 1
     assert lib.pgd_set_decode_math(0) == OK and lib.pgd_get_decode_math() == 0
+
+
+def test_wait_limit_hook_is_host_only(lib):
+    lib.pgd_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.pgd_debug_get_wait_limit_ns.restype = ctypes.c_uint64
+    assert lib.pgd_debug_get_wait_limit_ns() == 1_000_000_000
+    assert lib.pgd_debug_set_wait_limit_ns(5) == OK and lib.pgd_debug_get_wait_limit_ns() == 5
+    # 0 restores the default
+    assert lib.pgd_debug_set_wait_limit_ns(0) == OK
+    assert lib.pgd_debug_get_wait_limit_ns() == 1_000_000_000

@@ -66,6 +66,12 @@ MULTI = [  # (Hq, Hkv, D, bs, dtype, q_len)
     (8, 8, 128, 64, "bf16", 8), (16, 2, 128, 16, "bf16", 2), (12, 4, 128, 16, "bf16", 3),
     (8, 2, 256, 32, "bf16", 4), (4, 4, 256, 16, "bf16", 5), (32, 8, 128, 16, "e4m3", 4),
     (16, 8, 128, 64, "e4m3", 8), (8, 1, 128, 32, "e4m3", 2),
+    # 17 to 32 rows per KV head: two row groups of consumer warps, one pass
+    # over K/V (Llama shape g 4 with q_len 5-8; g 8 with q_len 3-4; g 16 at
+    # head_dim 256 with q_len 2)
+    (32, 8, 128, 16, "bf16", 8), (32, 8, 128, 16, "bf16", 5), (64, 8, 128, 64, "bf16", 4),
+    (64, 8, 128, 16, "e4m3", 4), (24, 8, 128, 32, "e4m3", 7), (32, 2, 256, 32, "bf16", 2),
+    (16, 2, 256, 16, "bf16", 3), (20, 4, 128, 64, "bf16", 6), (8, 1, 128, 16, "bf16", 3),
 ]
 
 
@@ -92,11 +98,29 @@ def test_sliding_window_multi_token(L, W):
     check_multi(w, multi_q(len(CTX), L, 8, 128, seed=951), W)
 
 
+@pytest.mark.parametrize("Hq,Hkv,D,bs,dt,L,W", [
+    (32, 8, 128, 16, "bf16", 8, 33), (64, 8, 128, 16, "e4m3", 4, 100),
+    (32, 2, 256, 32, "bf16", 2, 1000), (32, 8, 128, 64, "bf16", 8, 1)])
+def test_sliding_window_32_rows(Hq, Hkv, D, bs, dt, L, W):
+    w = make_case(CTX, Hq, Hkv, D, bs, dt, seed=955 + L + W, name=f"window-32rows-{dt}")
+    check_multi(w, multi_q(len(CTX), L, Hq, D, seed=956), W)
+
+
 @pytest.mark.parametrize("num_ctas", [1, 3, 29, 148, 1000])
 def test_multi_window_split_count_invariance(num_ctas):
     w = make_case([5000, 17, 640, 1, 0, 2222], 8, 2, 128, 16, "bf16", seed=960,
                   name="multi-split")
     check_multi(w, multi_q(6, 4, 8, 128, seed=961), 300, num_ctas=num_ctas)
+
+
+@pytest.mark.parametrize("num_ctas", [1, 7, 296, 1000])
+def test_32_rows_split_count_invariance(num_ctas):
+    """32 rows per KV head (g 4, q_len 8): units split over many CTAs are
+    merged by the two-pass column loop of the split merge."""
+    w = make_case([5000, 17, 640, 1, 0, 2222], 32, 8, 128, 16, "bf16", seed=962,
+                  name="multi-split-32")
+    check_multi(w, multi_q(6, 8, 32, 128, seed=963), 0, num_ctas=num_ctas)
+    check_multi(w, multi_q(6, 8, 32, 128, seed=964), 300, num_ctas=num_ctas)
 
 
 def test_single_token_no_window_is_the_plain_decode():
@@ -138,8 +162,30 @@ def test_window_never_reads_blocks_before_it():
 
 def test_multi_token_full_size_long_context():
     """A long-context batch at the sizes of the decode benchmark's long case,
-    four query tokens per sequence, g * q_len = 16 rows per KV head."""
+    four query tokens per sequence, g * q_len = 16 rows per KV head, and
+    eight (32 rows)."""
     ctx = [32768, 16384, 8192, 4096, 1, 31999]
     w = make_case(ctx, 32, 8, 128, 16, "bf16", seed=980, name="multi-long")
     check_multi(w, multi_q(len(ctx), 4, 32, 128, seed=981), 0)
     check_multi(w, multi_q(len(ctx), 4, 32, 128, seed=982), 4096)
+    check_multi(w, multi_q(len(ctx), 8, 32, 128, seed=983), 0)
+    check_multi(w, multi_q(len(ctx), 8, 32, 128, seed=984), 4096)
+
+
+def test_32_rows_repeat_and_permutation_bits():
+    """Two row groups merge in a fixed order: repeated runs, and the same
+    blocks placed elsewhere in the pool, give identical bits."""
+    w = make_case([3000, 700, 65, 1], 32, 8, 128, 16, "bf16", seed=985, name="multi-bits")
+    qm = multi_q(4, 8, 32, 128, seed=986)
+    d = Dev(w)
+    a, la = run_ex(d, qm, 0, num_ctas=41)
+    b, lb = run_ex(d, qm, 0, num_ctas=41)
+    assert np.array_equal(host_bits(a), host_bits(b)) and torch.equal(la, lb)
+    rng = np.random.default_rng(987)
+    perm = rng.permutation(w.num_blocks)
+    k2 = np.empty_like(w.k_cache)
+    v2 = np.empty_like(w.v_cache)
+    k2[perm], v2[perm] = w.k_cache, w.v_cache
+    w.k_cache, w.v_cache, w.block_table = k2, v2, perm[w.block_table].astype(np.int32)
+    c, lc = run_ex(Dev(w), qm, 0, num_ctas=41)
+    assert np.array_equal(host_bits(a), host_bits(c)) and torch.equal(la, lc)

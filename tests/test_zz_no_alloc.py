@@ -44,10 +44,18 @@ def test_noalloc_matches_allocating_entry_point_twice(ctx, Hq, Hkv, D, bs, dt):
     for call in range(2):
         lse = torch.full((w.num_seqs, Hq), float("nan"), dtype=torch.float32, device="cuda")
         out = torch.full_like(d.q, float("nan"))
+        torch.cuda.synchronize()
+        free_before = torch.cuda.mem_get_info()[0]
         pgd.paged_decode_attention_noalloc(d.q, d.k, d.v, d.bt, d.cl, Hq, Hkv, D, bs, w.scale,
                                            out, max_context_len=w.max_context_len,
                                            k_scale=d.ks, v_scale=d.vs, lse_out=lse)
         torch.cuda.synchronize()
+        free_after = torch.cuda.mem_get_info()[0]
+        if call == 1:
+            # the first call on a device may commit the static array; from
+            # then on a call leaves the device's free memory as it was
+            assert free_after == free_before, \
+                f"noalloc call changed free device memory by {free_before - free_after} bytes"
         got = to_f64(out)
         assert np.all(np.isfinite(got)), f"call {call}: non-finite output"
         assert_close(got, ref, dt, f"noalloc call {call}")
