@@ -5,6 +5,10 @@ device, checks their dtype/shape/contiguity, and passes raw pointers and the
 current stream to the C ABI declared in include/pgd.h.  All computation runs
 in the library's CUDA kernels; there is no fallback path.  If libpgd.so has
 not been built, loading raises ImportError.
+
+Every function that enqueues work also takes prepare=True: it then checks
+and marshals its arguments once and returns a Prepared call that re-issues
+the same C call (same buffers, sizes and stream) each time it is called.
 """
 from __future__ import annotations
 
@@ -105,6 +109,40 @@ def _check(status: int, where: str):
         raise PGDError(status, where)
 
 
+class Prepared:
+    """One library call with its arguments checked and marshalled once.
+
+    A serving loop issues the same call with the same buffers every step
+    (persistent q / out / cache tensors whose contents change); the
+    per-call checks and the conversion of ~25 arguments to C types then cost
+    more host time than a small batch's kernel takes on the GPU.  Calling a
+    Prepared object re-issues the C call with the pointers, sizes and stream
+    it was prepared with and returns what the original call returned.  The
+    tensors must stay alive and keep their storage while it is in use."""
+
+    __slots__ = ("_fn", "_args", "_name", "result")
+
+    def __init__(self, fn, args, name, result):
+        conv = []
+        for t, a in zip(fn.argtypes, args):
+            conv.append(a if a is None or isinstance(a, t) else t(a))
+        self._fn, self._args, self._name, self.result = fn, tuple(conv), name, result
+
+    def __call__(self):
+        st = self._fn(*self._args)
+        if st:
+            raise PGDError(st, self._name)
+        return self.result
+
+
+def _issue(fn, name: str, args, prepare: bool, result=None):
+    """Run the C call now, or return it prepared (see Prepared)."""
+    if prepare:
+        return Prepared(fn, args, name, result)
+    _check(fn(*args), name)
+    return result
+
+
 def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -139,7 +177,7 @@ def _need(t: torch.Tensor, name: str, dtypes, dim: Optional[int] = None):
 _KV_DTYPES = (torch.bfloat16, torch.uint8, torch.float8_e4m3fn)
 
 
-def kv_append(k_new, v_new, slot_mapping, k_cache, v_cache, *, stream=None) -> None:
+def kv_append(k_new, v_new, slot_mapping, k_cache, v_cache, *, stream=None, prepare=False):
     """Scatter new tokens' K/V rows into their cache slots (pgd_kv_append).
 
     k_new/v_new [N][Hkv][D] and caches [num_blocks][Hkv][bs][D] share one
@@ -155,9 +193,9 @@ def kv_append(k_new, v_new, slot_mapping, k_cache, v_cache, *, stream=None) -> N
     if v_cache.shape != k_cache.shape or k_new.shape != v_new.shape or \
             k_new.shape[1:] != (hkv, d) or slot_mapping.shape[0] != k_new.shape[0]:
         raise ValueError("kv_append: inconsistent shapes")
-    _check(lib.pgd_kv_append(_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), k_new.shape[0],
-                             _ptr(k_cache), _ptr(v_cache), hkv, d, bs, nb, _kv_dtype(k_cache),
-                             _stream(stream)), "pgd_kv_append")
+    return _issue(lib.pgd_kv_append, "pgd_kv_append",
+                  (_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), k_new.shape[0], _ptr(k_cache),
+                   _ptr(v_cache), hkv, d, bs, nb, _kv_dtype(k_cache), _stream(stream)), prepare)
 
 
 def kv_append_quant(k_new, v_new, slot_mapping, k_cache, v_cache, k_scale, v_scale, *,
@@ -192,7 +230,7 @@ def paged_decode_attention(q, k_cache, v_cache, block_table, context_lens, num_q
                            num_kv_heads: int, head_dim: int, block_size: int, scale: float,
                            out: Optional[torch.Tensor] = None, *, max_context_len: int = 0,
                            k_scale=None, v_scale=None, lse_out=None, workspace=None,
-                           num_ctas: int = 0, stream=None) -> torch.Tensor:
+                           num_ctas: int = 0, stream=None, prepare=False):
     """One decode step of paged GQA attention (pgd_paged_decode_attention).
 
     q bf16 [B][Hq][D]; caches [num_blocks][Hkv][bs][D] (bf16 or E4M3 bytes);
@@ -224,20 +262,18 @@ def paged_decode_attention(q, k_cache, v_cache, block_table, context_lens, num_q
     if workspace is not None:
         _need(workspace, "workspace", None)
         ws_bytes = workspace.numel() * workspace.element_size()
-    _check(lib.pgd_paged_decode_attention(
+    return _issue(lib.pgd_paged_decode_attention, "pgd_paged_decode_attention", (
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), block_table.shape[1],
         _ptr(context_lens), B, int(max_context_len), num_q_heads, num_kv_heads, head_dim,
         block_size, k_cache.shape[0], float(scale), kvd, _ptr(k_scale), _ptr(v_scale), _ptr(out),
-        _ptr(lse_out), _ptr(workspace), ws_bytes, int(num_ctas), _stream(stream)),
-        "pgd_paged_decode_attention")
-    return out
+        _ptr(lse_out), _ptr(workspace), ws_bytes, int(num_ctas), _stream(stream)), prepare, out)
 
 
 def paged_decode_attention_ex(q, k_cache, v_cache, block_table, context_lens, num_q_heads: int,
                               num_kv_heads: int, head_dim: int, block_size: int, scale: float,
                               out: Optional[torch.Tensor] = None, *, window: int = 0,
                               max_context_len: int = 0, k_scale=None, v_scale=None, lse_out=None,
-                              workspace=None, num_ctas: int = 0, stream=None) -> torch.Tensor:
+                              workspace=None, num_ctas: int = 0, stream=None, prepare=False):
     """Decode attention for q_len query tokens per sequence with an optional
     sliding window (pgd_paged_decode_attention_ex).
 
@@ -271,13 +307,12 @@ def paged_decode_attention_ex(q, k_cache, v_cache, block_table, context_lens, nu
     if workspace is not None:
         _need(workspace, "workspace", None)
         ws_bytes = workspace.numel() * workspace.element_size()
-    _check(lib.pgd_paged_decode_attention_ex(
+    return _issue(lib.pgd_paged_decode_attention_ex, "pgd_paged_decode_attention_ex", (
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), block_table.shape[1],
         _ptr(context_lens), B, int(max_context_len), L, int(window), num_q_heads, num_kv_heads,
         head_dim, block_size, k_cache.shape[0], float(scale), kvd, _ptr(k_scale), _ptr(v_scale),
         _ptr(out), _ptr(lse_out), _ptr(workspace), ws_bytes, int(num_ctas), _stream(stream)),
-        "pgd_paged_decode_attention_ex")
-    return out
+        prepare, out)
 
 
 def paged_decode_partial(q, k_cache, v_cache, block_table, context_lens, num_q_heads: int,
@@ -285,7 +320,7 @@ def paged_decode_partial(q, k_cache, v_cache, block_table, context_lens, num_q_h
                          o_part: Optional[torch.Tensor] = None,
                          lse_part: Optional[torch.Tensor] = None, *, max_context_len: int = 0,
                          k_scale=None, v_scale=None, workspace=None, num_ctas: int = 0,
-                         stream=None):
+                         stream=None, prepare=False):
     """Decode of one KV slice left unrounded for a merge
     (pgd_paged_decode_partial): returns (o_part fp32 [B][Hq][D],
     lse_part fp32 [B][Hq], natural log)."""
@@ -316,13 +351,12 @@ def paged_decode_partial(q, k_cache, v_cache, block_table, context_lens, num_q_h
     if workspace is not None:
         _need(workspace, "workspace", None)
         ws_bytes = workspace.numel() * workspace.element_size()
-    _check(lib.pgd_paged_decode_partial(
+    return _issue(lib.pgd_paged_decode_partial, "pgd_paged_decode_partial", (
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), block_table.shape[1],
         _ptr(context_lens), B, int(max_context_len), num_q_heads, num_kv_heads, head_dim,
         block_size, k_cache.shape[0], float(scale), kvd, _ptr(k_scale), _ptr(v_scale),
         _ptr(o_part), _ptr(lse_part), _ptr(workspace), ws_bytes, int(num_ctas), _stream(stream)),
-        "pgd_paged_decode_partial")
-    return o_part, lse_part
+        prepare, (o_part, lse_part))
 
 
 _MATH = {"tensor_core": 0, "cuda_core": 1}
@@ -372,7 +406,7 @@ def decode_step(q, k_new, v_new, k_cache, v_cache, block_table, context_lens, nu
                 num_kv_heads: int, head_dim: int, block_size: int, scale: float,
                 out: Optional[torch.Tensor] = None, *, max_context_len: int = 0, k_scale=None,
                 v_scale=None, lse_out=None, workspace=None, num_ctas: int = 0,
-                stream=None) -> torch.Tensor:
+                stream=None, prepare=False):
     """One decode step in one launch (pgd_decode_step): writes each sequence's
     newest K/V row (k_new / v_new [B][Hkv][D], cache dtype) at position
     context_lens[s] - 1, then computes paged decode attention over the
@@ -404,13 +438,12 @@ def decode_step(q, k_new, v_new, k_cache, v_cache, block_table, context_lens, nu
     if workspace is not None:
         _need(workspace, "workspace", None)
         ws_bytes = workspace.numel() * workspace.element_size()
-    _check(lib.pgd_decode_step(
+    return _issue(lib.pgd_decode_step, "pgd_decode_step", (
         _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
         block_table.shape[1], _ptr(context_lens), B, int(max_context_len), num_q_heads,
         num_kv_heads, head_dim, block_size, k_cache.shape[0], float(scale), kvd, _ptr(k_scale),
         _ptr(v_scale), _ptr(out), _ptr(lse_out), _ptr(workspace), ws_bytes, int(num_ctas),
-        _stream(stream)), "pgd_decode_step")
-    return out
+        _stream(stream)), prepare, out)
 
 
 def paged_decode_attention_noalloc(q, k_cache, v_cache, block_table, context_lens,
@@ -452,7 +485,7 @@ def paged_decode_attention_noalloc(q, k_cache, v_cache, block_table, context_len
     return out
 
 
-def merge_partials(o_part, lse_part, out=None, lse_out=None, *, stream=None) -> torch.Tensor:
+def merge_partials(o_part, lse_part, out=None, lse_out=None, *, stream=None, prepare=False):
     """LSE merge of split results: o_part fp32 [P][rows][D], lse_part fp32
     [P][rows] (natural log) -> out bf16 [rows][D] (pgd_merge_partials)."""
     lib = load_library()
@@ -466,9 +499,9 @@ def merge_partials(o_part, lse_part, out=None, lse_out=None, *, stream=None) -> 
     _need(out, "out", (torch.bfloat16,), 2)
     if lse_out is not None:
         _need(lse_out, "lse_out", (torch.float32,), 1)
-    _check(lib.pgd_merge_partials(_ptr(o_part), _ptr(lse_part), P, R, D, _ptr(out),
-                                  _ptr(lse_out), _stream(stream)), "pgd_merge_partials")
-    return out
+    return _issue(lib.pgd_merge_partials, "pgd_merge_partials",
+                  (_ptr(o_part), _ptr(lse_part), P, R, D, _ptr(out), _ptr(lse_out),
+                   _stream(stream)), prepare, out)
 
 
 def get_device_error(*, stream=None) -> int:

@@ -86,6 +86,8 @@ struct DecodeParams {
     // limit of every pipeline wait in ns (kDefaultWaitNs unless a test of
     // the timeout path shortens it)
     uint64_t wait_ns;
+    // 1: a whole unit that fits in one stage goes to one consumer warp alone
+    int32_t short_units;
 };
 
 constexpr int kConsumerWarps = 4;
@@ -98,12 +100,16 @@ constexpr float kLn2 = 0.6931471805599453f;
 // moves a row's reference max (lazy rescaling)
 constexpr float kLazyRescale = 8.f;
 constexpr uint32_t kBarConsumers = 1;
+// segment kinds (SegDesc::kind); 0 .. 3 name the one consumer warp that
+// processes a short unit alone
+constexpr int kSegTerminal = -1;   // no more segments for this CTA
+constexpr int kSegShared = 4;      // every consumer warp takes a share of the tokens
 
 // Segment descriptor written by the producer, read by the consumers.
 struct SegDesc {
     long long u;      // flattened index of the segment's first tile
     int s, h, j0, j1, n, ctx;
-    int terminal;     // 1: no more segments for this CTA
+    int kind;         // kSegTerminal, kSegShared, or the warp of a short unit
     float ksc, vsc;   // FP8 per-KV-head scales (1 for bf16)
     int jlo;          // first block any query row of the unit sees
 };
@@ -132,11 +138,20 @@ struct DecodeCfg {
     static constexpr int DT = D / 16;                    // PV m-tiles (each warp: all of D)
     static constexpr int KSTEPS = D / 16;                // QK k-steps
     // head_dim 256 with tensor cores: the query rows stay in shared memory
-    // for the whole segment (row stride padded by 16 bytes so that an
-    // ldmatrix of 8 rows hits 8 bank groups) instead of in registers
+    // for the whole segment (read by ldmatrix) instead of in registers
     static constexpr bool QSMEM = D == 256 && !FP8 && CC == 0;
-    static constexpr int QROW = QSMEM ? D * 2 + 16 : D * 2;
+    // The tensor-core consumers' query slot pads each row, so that the 8 rows
+    // a fragment load touches fall in different banks: 16 bytes for bf16
+    // (4-byte loads, and ldmatrix at head_dim 256), 32 bytes for FP8 (one
+    // 8-byte load per k-step).  Each row then arrives by its own bulk copy.
+    static constexpr bool QPAD = CC == 0;
+    static constexpr int QROW = QPAD ? D * 2 + (FP8 ? 32 : 16) : D * 2;
     static constexpr int QSLOT = NP * QROW;              // query rows of one unit
+    // Short units (whole in the CTA, at most one stage of tiles) may go to one
+    // consumer warp each, which then needs every row of the unit in its own
+    // registers: up to 8 rows, query fragments held in registers (the 16-row
+    // variant has no registers to spare for the extra output path).
+    static constexpr bool SHORT = CC == 0 && NT == 1 && !QSMEM;
     // descriptor ring depth (one slot for 16 or more query rows at head_dim
     // 128, so that two CTAs still fit on an SM; one for 32 rows at 256)
     static constexpr int NSEG =
@@ -645,6 +660,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         Cursor cur = first_unit<BS>(p, misc->s0, misc->pfx0, u0, win0);
         const uint32_t qtok = (uint32_t)(g * D * 2);          // one query token's rows
         uint32_t it = 0, sit = 0, ait = 0;
+        uint32_t nshort = 0;                                  // short units so far
         bool ok = true;
         // FP8 scales of the first 32 KV heads, one per lane
         float ks_l = 1.f, vs_l = 1.f;
@@ -696,6 +712,13 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     vsc = __ldg(p.v_scale + cur.h);
                 }
             }
+            // A whole unit whose tiles fit in one stage goes to one consumer
+            // warp alone, round robin over the CTA's short units: the four
+            // warps then work on four units at once, and none of them waits
+            // for a merge across warps.
+            int kind = kSegShared;
+            if (C::SHORT && p.short_units && j0 == cur.jlo && j1 == cur.n && j1 - j0 <= C::BPS)
+                kind = (int)(nshort++ & 3u);
             // -- descriptor and query rows of the segment
             {
                 const uint32_t slot = sit % C::NSEG;
@@ -712,21 +735,21 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     d.j1 = j1;
                     d.n = cur.n;
                     d.ctx = cur.ctx;
-                    d.terminal = 0;
+                    d.kind = kind;
                     d.ksc = ksc;
                     d.vsc = vsc;
                     d.jlo = cur.jlo;
                     const uint32_t bar = seg_full + 8 * slot;
                     mbar_arrive_expect_tx(bar, qtok * p.q_len);
                     // query rows: q_len runs of g contiguous heads, row = i*g + head
-                    if (!C::QSMEM)
+                    if (!C::QPAD)
                         for (int i = 0; i < p.q_len; ++i)
                             bulk_copy_g2s(sQ + slot * C::QSLOT + i * qtok,
                                           p.q + (((long long)cur.s * p.q_len + i) * p.num_q_heads +
                                                  (long long)cur.h * g) * D,
                                           qtok, bar);
                 }
-                if (C::QSMEM) {
+                if (C::QPAD) {
                     // one copy per row into the padded slot (after the expect-tx)
                     __syncwarp();
                     for (int r = lane; r < g * p.q_len; r += 32)
@@ -811,7 +834,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     raise_flag(p.flags, kFlagTimeout);
             // terminal descriptor (also after a timeout, so that the consumers stop)
             if (free_slot) {
-                segs[slot].terminal = 1;
+                segs[slot].kind = kSegTerminal;
                 mbar_arrive(seg_full + 8 * slot);
             }
         }
@@ -835,11 +858,17 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         const int j1 = (int)lds32(da + offsetof(SegDesc, j1));
         const int nunit = (int)lds32(da + offsetof(SegDesc, n));
         const int ctx = (int)lds32(da + offsetof(SegDesc, ctx));
-        const int terminal = (int)lds32(da + offsetof(SegDesc, terminal));
+        const int kind = (int)lds32(da + offsetof(SegDesc, kind));
         const float ksc = __uint_as_float(lds32(da + offsetof(SegDesc, ksc)));
         const float vsc = __uint_as_float(lds32(da + offsetof(SegDesc, vsc)));
         const int jlo = (int)lds32(da + offsetof(SegDesc, jlo));
-        if (named_bar_sync_or(kBarConsumers, kConsumers, !seg_ok || terminal)) return;
+        // A short unit belongs to one warp and needs no barrier.  Every other
+        // segment (and a wait that timed out, whose descriptor may be stale)
+        // meets all consumer warps at a barrier that also agrees on leaving.
+        const bool alone = C::SHORT && seg_ok && kind >= 0 && kind < kSegShared;
+        if (!alone &&
+            named_bar_sync_or(kBarConsumers, kConsumers, !seg_ok || kind == kSegTerminal))
+            return;
         const bool whole = (j0 == jlo && j1 == nunit);
         const int R = p.rows;
 
@@ -898,6 +927,25 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         };
 
         if constexpr (CC == 0) {
+            if (alone && warp != kind) {
+                // another warp's short unit: free the descriptor slot, and its
+                // one stage once it has landed (so that this warp's arrivals
+                // stay in step with the ring's phases)
+                __syncwarp();
+                if (lane == 0) mbar_arrive(seg_empty + 8 * qs);
+                ++sit;
+                const uint32_t slot = it % NSTAGES;
+                const bool ok = mbar_wait_bounded(bar_full + 8 * slot, (it / NSTAGES) & 1, p.wait_ns);
+                ++it;
+                if (!ok) {
+                    raise_flag(p.flags, kFlagTimeout);
+                    named_bar_sync_or(kBarConsumers, kConsumers, true);   // leave with the others
+                    return;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_empty + 8 * slot);
+                continue;
+            }
             // This warp's row group: rows rbase .. rbase + 8 * NTW - 1 (all rows
             // unless the unit has 32, when warps 0, 1 take rows 0-15 and warps 2,
             // 3 rows 16-31)
@@ -927,16 +975,18 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 for (int nt = 0; nt < C::NTW; ++nt) {
                     const int head = rbase + nt * 8 + gid;   // query row held as B column
                     const bool live = head < R;
-                    const uint32_t qr = qb + (live ? head : 0) * D * 2;
+                    const uint32_t qr = qb + (live ? head : 0) * C::QROW;
 #pragma unroll
                     for (int k = 0; k < C::KSTEPS; ++k) {
                         uint32_t b0, b1;
                         if (!FP8) {   // k index 2t, 2t+1 | 2t+8, 2t+9  <->  same d
                             b0 = lds32(qr + (16 * k + 2 * t4) * 2);
                             b1 = lds32(qr + (16 * k + 8 + 2 * t4) * 2);
-                        } else {      // k index permuted to d = 16k + 4t + {0,1 | 2,3}
-                            b0 = lds32(qr + (16 * k + 4 * t4) * 2);       // bf16 pairs,
-                            b1 = lds32(qr + (16 * k + 4 * t4 + 2) * 2);   // converted below
+                        } else {      // k index permuted to d = 16k + 4t + {0,1 | 2,3}:
+                            // 4 consecutive bf16, converted to f16 below
+                            const long long v = lds64(qr + (16 * k + 4 * t4) * 2);
+                            b0 = (uint32_t)v;
+                            b1 = (uint32_t)((unsigned long long)v >> 32);
                         }
                         qf[k][nt][0] = live ? b0 : 0u;
                         qf[k][nt][1] = live ? b1 : 0u;
@@ -1016,9 +1066,13 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 }
                 const uint32_t sK = sbase + slot * C::STAGE, sV = sK + C::STAGE_KV;
 
-                for (int sub = 0; sub < C::SUBS; ++sub) {
+                // 16-token sub-tiles of this warp: its own 16 (or 32) tokens of
+                // the stage, or every token of a short unit it holds alone
+                const int nsub = alone ? (n_valid + 15) / 16 : C::SUBS;
+                for (int sub = 0; sub < nsub; ++sub) {
                     // first stage token of this warp's 16-token sub-tile
-                    const int tb = C::RG == 1 ? 16 * warp : 32 * (warp & 1) + 16 * sub;
+                    const int tb = alone ? 16 * sub
+                                         : (C::RG == 1 ? 16 * warp : 32 * (warp & 1) + 16 * sub);
                     if (tb < n_valid) {
                         // ---- S^T = K . Q^T for this warp's 16 tokens (two MMA chains)
                         float sacc[C::NTW][4], sac2[C::NTW][4];
@@ -1257,6 +1311,73 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 if (!FP8) return 16 * mt + gid + (e >> 1) * 8;
                 return 16 * gid + 2 * mt + (e >> 1);
             };
+            if (alone) {
+                // The warp holds the short unit's whole softmax state: out (or the
+                // fp32 result) and lse go straight from its accumulators.
+                if (abort) {
+                    named_bar_sync_or(kBarConsumers, kConsumers, true);   // leave with the others
+                    return;
+                }
+                float inv[C::NTW][2];
+#pragma unroll
+                for (int nt = 0; nt < C::NTW; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        float l = l_run[nt][e];
+#pragma unroll
+                        for (int off = 4; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+                        inv[nt][e] = l > 0.f ? vsc / l : 0.f;
+                        const int r = nt * 8 + 2 * t4 + e;
+                        if (p.lse_out && gid == 0 && r < R)
+                            p.lse_out[orow(r)] = l > 0.f ? (m_run[nt][e] + log2f(l)) * kLn2 : -INFINITY;
+                    }
+                if (p.out_f32) {
+                    float *of = reinterpret_cast<float *>(p.out);
+#pragma unroll
+                    for (int mt = 0; mt < C::DT; ++mt)
+#pragma unroll
+                        for (int nt = 0; nt < C::NTW; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int r = nt * 8 + 2 * t4 + (e & 1);
+                                if (r < R) of[orow(r) * D + dim_of(mt, e)] = o[mt][nt][e] * inv[nt][e & 1];
+                            }
+                } else if constexpr (!FP8) {
+                    // a warp transpose of each 8x8 half gives lane (gid, t4) query
+                    // row 8nt + gid at dims 16mt + 8hf + 2t4 and the next one
+#pragma unroll
+                    for (int mt = 0; mt < C::DT; ++mt)
+#pragma unroll
+                        for (int nt = 0; nt < C::NTW; ++nt)
+#pragma unroll
+                            for (int hf = 0; hf < 2; ++hf) {
+                                const uint32_t t = movmatrix_trans(
+                                    pack_bf16x2(o[mt][nt][2 * hf] * inv[nt][0],
+                                                o[mt][nt][2 * hf + 1] * inv[nt][1]));
+                                const int r = nt * 8 + gid;
+                                if (r < R)
+                                    *reinterpret_cast<uint32_t *>(p.out + orow(r) * D + 16 * mt +
+                                                                  8 * hf + 2 * t4) = t;
+                            }
+                } else {
+                    // FP8 layout: elements c and c + 2 are dims 16gid + 2mt and the
+                    // next one of query row 8nt + 2t4 + c
+#pragma unroll
+                    for (int mt = 0; mt < C::DT; ++mt)
+#pragma unroll
+                        for (int nt = 0; nt < C::NTW; ++nt)
+#pragma unroll
+                            for (int c = 0; c < 2; ++c) {
+                                const int r = nt * 8 + 2 * t4 + c;
+                                if (r < R)
+                                    *reinterpret_cast<uint32_t *>(p.out + orow(r) * D + 16 * gid +
+                                                                  2 * mt) =
+                                        pack_bf16x2(o[mt][nt][c] * inv[nt][c],
+                                                    o[mt][nt][c + 2] * inv[nt][c]);
+                            }
+                }
+                continue;
+            }
             // A: warps 0, 1; B: warps 2, 3
             auto store_rows = [&](int nt) {
                 float *buf = reinterpret_cast<float *>(

@@ -377,3 +377,30 @@ def test_quantised_append_then_fp8_decode():
     w.k_cache, w.v_cache = ek, ev
     ref, _ = oracle_full(w)
     assert_close(to_f64(out), ref, "e4m3", "quantised append + decode")
+
+
+# --------------------------------------------------------------------------- #
+# prepared calls: the same C call re-issued with the arguments marshalled once
+# --------------------------------------------------------------------------- #
+def test_prepared_calls_give_the_same_bits():
+    w = make_case([1, 17, 64, 200, 999], 32, 8, 128, 16, "bf16", seed=19, append_last=True)
+    kn, vn = _step_payload(w)
+    from tests.gpu_helpers import dev_cache
+    d1, d2 = Dev(w), Dev(w)
+    kn_d, vn_d = dev_cache(kn), dev_cache(vn)
+    out1 = pgd.decode_step(d1.q, kn_d, vn_d, d1.k, d1.v, d1.bt, d1.cl, 32, 8, 128, 16, w.scale,
+                           max_context_len=w.max_context_len)
+    out2 = torch.empty_like(out1)
+    call = pgd.decode_step(d2.q, kn_d, vn_d, d2.k, d2.v, d2.bt, d2.cl, 32, 8, 128, 16, w.scale,
+                           out2, max_context_len=w.max_context_len, prepare=True)
+    for _ in range(3):
+        assert call() is out2
+    torch.cuda.synchronize()
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    # the prepared call reads the buffers' current contents on every call
+    d2.q.copy_(d2.q.flip(0))
+    call()
+    out3 = pgd.decode_step(d1.q.flip(0).contiguous(), kn_d, vn_d, d1.k, d1.v, d1.bt, d1.cl, 32,
+                           8, 128, 16, w.scale, max_context_len=w.max_context_len)
+    torch.cuda.synchronize()
+    assert torch.equal(out2.view(torch.int16), out3.view(torch.int16))
