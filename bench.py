@@ -426,6 +426,90 @@ def mode_kvp(args, w, pgd, dev, stream, rank, world):
     return m
 
 
+def mode_op(args, w, pgd, dev, stream):
+    """One auxiliary kernel alone, on the workload's shapes:
+      kv_append        N new tokens' bf16 (or E4M3) K/V rows scattered into
+                       N distinct cache slots (pgd_kv_append)
+      kv_append_quant  N bf16 rows quantised into an E4M3 cache
+                       (pgd_kv_append_quant)
+      merge            the log-sum-exp merge of P split results of every
+                       (sequence, query head) row (pgd_merge_partials)
+    N = --append-tokens (default: one per sequence); P = --merge-parts."""
+    import torch
+    m = Mode()
+    rng = np.random.default_rng(77)
+    Hkv, D, bs = w.num_kv_heads, w.head_dim, w.block_size
+    if args.op in ("kv_append", "kv_append_quant"):
+        N = args.append_tokens or w.num_seqs
+        pool = max(w.num_blocks, -(-N // bs))
+        if args.op == "kv_append":
+            e = w.elem_bytes
+            dt = torch.bfloat16 if e == 2 else torch.uint8
+        else:
+            e, dt = 1, torch.uint8
+        k = torch.zeros((pool, Hkv, bs, D), dtype=dt, device=dev)
+        v = torch.zeros_like(k)
+        src_dt = torch.bfloat16 if args.op == "kv_append_quant" else dt
+        host = {"kn": torch.randn((N, Hkv, D)).to(src_dt) if src_dt == torch.bfloat16 else
+                torch.randint(0, 120, (N, Hkv, D), dtype=torch.uint8),
+                "sl": torch.from_numpy(rng.permutation(pool * bs)[:N].astype(np.int64))}
+        host["vn"] = host["kn"].flip(0).contiguous()
+        ks = torch.full((Hkv,), 0.01, dtype=torch.float32, device=dev)
+        m.inputs = {n: t.to(dev) for n, t in host.items()}
+        m.host = {n: t.pin_memory() for n, t in host.items()}
+        m.out = k
+        src_e = 2 if args.op == "kv_append_quant" else e
+        m.dec_bytes = m.step_bytes = 2 * N * Hkv * D * (src_e + e) + 8 * N + \
+            (8 * Hkv if args.op == "kv_append_quant" else 0)
+        m.read_bytes = 2 * N * Hkv * D * src_e
+        prepared = {}
+
+        def step(inp, ev=None, r=0):
+            key = id(inp)
+            if key not in prepared:
+                if args.op == "kv_append":
+                    prepared[key] = pgd.kv_append(inp["kn"], inp["vn"], inp["sl"], k, v,
+                                                  stream=stream, prepare=True)
+                else:
+                    prepared[key] = pgd.kv_append_quant(inp["kn"], inp["vn"], inp["sl"], k, v,
+                                                        ks, ks, stream=stream, prepare=True)
+            if ev:
+                ev[0].record(stream)
+            prepared[key]()
+            if ev:
+                ev[1].record(stream)
+
+        m.kernel = "kv_append_kernel" if args.op == "kv_append" else "kv_append_quant_kernel"
+        m.cfg = {"op": args.op, "append_tokens": N, "pool_slots": pool * bs}
+    else:
+        P, rows = args.merge_parts, w.num_seqs * w.num_q_heads
+        host = {"o": torch.randn((P, rows, D), dtype=torch.float32),
+                "l": (torch.randn((P, rows), dtype=torch.float32) * 3)}
+        m.inputs = {n: t.to(dev) for n, t in host.items()}
+        m.host = {n: t.pin_memory() for n, t in host.items()}
+        m.out = torch.empty((rows, D), dtype=torch.bfloat16, device=dev)
+        m.dec_bytes = m.step_bytes = P * rows * (D + 1) * 4 + rows * D * 2
+        m.read_bytes = P * rows * (D + 1) * 4
+        prepared = {}
+
+        def step(inp, ev=None, r=0):
+            key = id(inp)
+            if key not in prepared:
+                prepared[key] = pgd.merge_partials(inp["o"], inp["l"], inp.get("out", m.out),
+                                                   stream=stream, prepare=True)
+            if ev:
+                ev[0].record(stream)
+            prepared[key]()
+            if ev:
+                ev[1].record(stream)
+
+        m.kernel = "merge_partials_kernel"
+        m.cfg = {"op": "merge", "merge_parts": P, "rows": rows}
+    m.step, m.single, m.launches, m.fused = step, True, 1, False
+    m.replicas = 1
+    return m
+
+
 def torch_empty_like(t):
     import torch
     return torch.empty_like(t)
@@ -450,7 +534,9 @@ def run_ours(args, rank, world, local_rank):
         # every rank runs its own batch: same shape (context lengths of seed
         # 0), its own block permutation and values
         w = make_workload(args.workload, seed=rank, shape_seed=0)
-        if args.q_len > 1 or args.window > 0:
+        if args.op:
+            m = mode_op(args, w, pgd, dev, stream)
+        elif args.q_len > 1 or args.window > 0:
             m = mode_ex(args, w, pgd, dev, stream)
         else:
             m = mode_step(args, w, pgd, dev, stream)
@@ -505,71 +591,80 @@ def run_ours(args, rank, world, local_rank):
     iso_ms = sum(a_.elapsed_time(b_) for a_, b_ in iso) / len(iso)
 
     # ---- end to end through the public API with host buffers ----------------
-    # Every step copies its inputs from pinned host memory (packed into one
-    # buffer, one copy) and reads its output back.  As in a serving loop, the
-    # input copy of step i+1 and the read-back of step i-1 run on their own
-    # streams while step i decodes (inputs and outputs double-buffered); all
-    # of every step's copies are inside the timed region.
-    names = list(m.host.keys())
-    nbytes = {n: m.host[n].numel() * m.host[n].element_size() for n in names}
-    offs, total = {}, 0
-    for n in names:
-        offs[n] = total
-        total += (nbytes[n] + 255) // 256 * 256
-    hpack = torch.empty(total, dtype=torch.uint8, pin_memory=True)
-    for n in names:
-        hpack[offs[n]:offs[n] + nbytes[n]].copy_(m.host[n].reshape(-1).view(torch.uint8))
-    dpack = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(2)]
-    bufs = []
-    for b in range(2):
-        views = {n: dpack[b][offs[n]:offs[n] + nbytes[n]].view(m.host[n].dtype)
-                 .view(m.host[n].shape) for n in names}
-        views["out"] = torch.empty_like(m.out)
-        bufs.append(views)
-    hout = [torch.empty(m.out.shape, dtype=m.out.dtype, pin_memory=True) for _ in range(2)]
-    s_h2d = torch.cuda.Stream(device=dev)
-    s_d2h = torch.cuda.Stream(device=dev)
-    ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of buffer b copied
-    ev_cmp = [torch.cuda.Event() for _ in range(2)]    # step using buffer b computed
-    ev_out = [torch.cuda.Event() for _ in range(2)]    # output of buffer b read back
-    h2d_bytes = total
-    d2h_bytes = hout[0].numel() * hout[0].element_size()
-    Ke = max(1, min(K, args.e2e_steps))
+    def e2e_run():
+        # Every step copies its inputs from pinned host memory (packed into one
+        # buffer, one copy) and reads its output back.  As in a serving loop, the
+        # input copy of step i+1 and the read-back of step i-1 run on their own
+        # streams while step i decodes (inputs and outputs double-buffered); all
+        # of every step's copies are inside the timed region.
+        names = list(m.host.keys())
+        nbytes = {n: m.host[n].numel() * m.host[n].element_size() for n in names}
+        offs, total = {}, 0
+        for n in names:
+            offs[n] = total
+            total += (nbytes[n] + 255) // 256 * 256
+        hpack = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+        for n in names:
+            hpack[offs[n]:offs[n] + nbytes[n]].copy_(m.host[n].reshape(-1).view(torch.uint8))
+        dpack = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(2)]
+        bufs = []
+        for b in range(2):
+            views = {n: dpack[b][offs[n]:offs[n] + nbytes[n]].view(m.host[n].dtype)
+                     .view(m.host[n].shape) for n in names}
+            views["out"] = torch.empty_like(m.out)
+            bufs.append(views)
+        hout = [torch.empty(m.out.shape, dtype=m.out.dtype, pin_memory=True) for _ in range(2)]
+        s_h2d = torch.cuda.Stream(device=dev)
+        s_d2h = torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of buffer b copied
+        ev_cmp = [torch.cuda.Event() for _ in range(2)]    # step using buffer b computed
+        ev_out = [torch.cuda.Event() for _ in range(2)]    # output of buffer b read back
+        h2d_bytes = total
+        d2h_bytes = hout[0].numel() * hout[0].element_size()
+        Ke = max(1, min(K, args.e2e_steps))
 
-    def e2e_steps(n):
-        for i in range(n):
-            b = i % 2
-            if i >= 2:
-                s_h2d.wait_event(ev_cmp[b])            # step i-2 no longer reads buffer b
-            with torch.cuda.stream(s_h2d):
-                dpack[b].copy_(hpack, non_blocking=True)
-            ev_in[b].record(s_h2d)
-            stream.wait_event(ev_in[b])
-            if i >= 2:
-                stream.wait_event(ev_out[b])           # output of step i-2 read back
-            m.step(bufs[b], None, i % R)
-            ev_cmp[b].record(stream)
-            s_d2h.wait_event(ev_cmp[b])
-            with torch.cuda.stream(s_d2h):
-                hout[b].copy_(bufs[b]["out"], non_blocking=True)
-            ev_out[b].record(s_d2h)
+        def e2e_steps(n):
+            for i in range(n):
+                b = i % 2
+                if i >= 2:
+                    s_h2d.wait_event(ev_cmp[b])            # step i-2 no longer reads buffer b
+                with torch.cuda.stream(s_h2d):
+                    dpack[b].copy_(hpack, non_blocking=True)
+                ev_in[b].record(s_h2d)
+                stream.wait_event(ev_in[b])
+                if i >= 2:
+                    stream.wait_event(ev_out[b])           # output of step i-2 read back
+                m.step(bufs[b], None, i % R)
+                ev_cmp[b].record(stream)
+                s_d2h.wait_event(ev_cmp[b])
+                with torch.cuda.stream(s_d2h):
+                    hout[b].copy_(bufs[b]["out"], non_blocking=True)
+                ev_out[b].record(s_d2h)
 
-    e2e_steps(3)
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    f0 = torch.cuda.Event(enable_timing=True)
-    f1 = torch.cuda.Event(enable_timing=True)
-    f0.record(s_h2d)
-    e2e_steps(Ke)
-    s_d2h.wait_event(ev_cmp[(Ke - 1) % 2])
-    f1.record(s_d2h)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = f0.elapsed_time(f1) / Ke
-    # the kernels are deterministic: the read-back output is the resident run's
-    assert torch.equal(hout[(Ke - 1) % 2].view(torch.uint8), m.out.cpu().view(torch.uint8)), \
-        "end-to-end output differs from the device-resident run"
+        e2e_steps(3)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(s_h2d)
+        e2e_steps(Ke)
+        s_d2h.wait_event(ev_cmp[(Ke - 1) % 2])
+        f1.record(s_d2h)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = f0.elapsed_time(f1) / Ke
+        # the kernels are deterministic: the read-back output is the resident run's
+        assert torch.equal(hout[(Ke - 1) % 2].view(torch.uint8), m.out.cpu().view(torch.uint8)), \
+            "end-to-end output differs from the device-resident run"
+        return e2e_ms, h2d_bytes, d2h_bytes, Ke
+
+    if args.op:
+        # an auxiliary kernel alone: no end-to-end line (its result is the
+        # cache or a merged output of other launches, not a step's output)
+        e2e_ms, h2d_bytes, d2h_bytes, Ke = float("nan"), 0, 0, 0
+    else:
+        e2e_ms, h2d_bytes, d2h_bytes, Ke = e2e_run()
 
     # ---- aggregate over ranks ----------------------------------------------------
     ms_step = ms_total / K
@@ -582,7 +677,7 @@ def run_ours(args, rank, world, local_rank):
 
     probe = copy_probe(dev) if not args.no_copy_probe else None
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.op:
         cpu = cpu_baseline(w, args.cpu_seconds)
 
     if rank == 0:
@@ -603,7 +698,7 @@ def run_ours(args, rank, world, local_rank):
                     f"replicas x{world} (independent batch per GPU)",
                     "l2": l2, "cache_copies": R,
                     "global_batch": w.num_seqs * (1 if args.kvp else world)})
-        default_mode = not args.kvp and args.q_len == 1 and args.window == 0
+        default_mode = not args.kvp and args.q_len == 1 and args.window == 0 and not args.op
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
@@ -633,7 +728,7 @@ def run_ours(args, rank, world, local_rank):
                     "steps": Ke,
                     "copies": "one packed H2D of the step's inputs and one D2H of its output "
                               "per step, on their own streams, overlapping the neighbouring "
-                              "steps' decode (double-buffered)"},
+                              "steps' decode (double-buffered)"} if not args.op else None,
             "gpu_launches": K * m.launches,
             "fused_step": m.fused,
             "clocks": clk,
@@ -764,6 +859,12 @@ def main():
                          "bf16 head_dim 128 with <= 8 query rows per KV head)")
     ap.add_argument("--kvp", action="store_true",
                     help="split every sequence's KV over the ranks (strong scaling)")
+    ap.add_argument("--op", choices=["kv_append", "kv_append_quant", "merge"], default=None,
+                    help="time one auxiliary kernel alone on the workload's shapes")
+    ap.add_argument("--append-tokens", type=int, default=0,
+                    help="--op kv_append*: new tokens per call (default: one per sequence)")
+    ap.add_argument("--merge-parts", type=int, default=8,
+                    help="--op merge: split results merged per row")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -771,6 +872,8 @@ def main():
         ap.error("--q-len must be >= 1 and --window >= 0")
     if args.kvp and (args.q_len > 1 or args.window > 0 or args.unfused):
         ap.error("--kvp runs the one-token decode without append")
+    if args.op and (args.kvp or args.q_len > 1 or args.window > 0 or args.unfused):
+        ap.error("--op times one auxiliary kernel alone")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
