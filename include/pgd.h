@@ -310,7 +310,7 @@ pgd_decode_math pgd_get_decode_math(void);
  * descriptor, a free ring slot, an appended row) is bounded: after the limit
  * the kernel raises the timeout flag (8), its warps leave together, the
  * producer still waits for every copy it issued (with its own fixed limit of
- * 0.2 s) so nothing lands after the CTA exits, and pgd_get_device_error()
+ * 1 s) so nothing lands after the CTA exits, and pgd_get_device_error()
  * returns PGD_ERR_TIMEOUT and re-zeroes the arrival counters, so the next
  * call starts clean.  No correct input makes a wait run out, so this hook
  * exists to test that path: a limit of a few ns makes the waits give up.
@@ -423,9 +423,9 @@ pgd_status pgd_paged_decode_attention_noalloc(
  * Splits with lse = -inf carry no weight; a row whose splits are all -inf
  * gives out = 0, lse = -inf.  Used to merge per-GPU splits of one sequence.
  *
- *   o_part    device fp32 [num_parts][rows][head_dim]
+ *   o_part    device fp32 [num_parts][rows][head_dim], 16-byte aligned
  *   lse_part  device fp32 [num_parts][rows] (natural log)
- *   out       device bf16 [rows][head_dim]
+ *   out       device bf16 [rows][head_dim], 8-byte aligned
  *   lse_out   optional device fp32 [rows], NULL to skip
  *   num_parts >= 1, rows >= 0, head_dim in {128, 256}
  */

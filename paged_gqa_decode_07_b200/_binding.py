@@ -199,7 +199,7 @@ def kv_append(k_new, v_new, slot_mapping, k_cache, v_cache, *, stream=None, prep
 
 
 def kv_append_quant(k_new, v_new, slot_mapping, k_cache, v_cache, k_scale, v_scale, *,
-                    stream=None) -> None:
+                    stream=None, prepare=False):
     """Quantise bf16 K/V rows of new tokens into an FP8 E4M3 cache
     (pgd_kv_append_quant): byte = E4M3(x / scale[kv head])."""
     lib = load_library()
@@ -215,9 +215,10 @@ def kv_append_quant(k_new, v_new, slot_mapping, k_cache, v_cache, k_scale, v_sca
             k_new.shape[1:] != (hkv, d) or slot_mapping.shape[0] != k_new.shape[0] or \
             k_scale.shape != (hkv,) or v_scale.shape != (hkv,):
         raise ValueError("kv_append_quant: inconsistent shapes")
-    _check(lib.pgd_kv_append_quant(_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), k_new.shape[0],
-                                   _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
-                                   hkv, d, bs, nb, _stream(stream)), "pgd_kv_append_quant")
+    return _issue(lib.pgd_kv_append_quant, "pgd_kv_append_quant",
+                  (_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), k_new.shape[0], _ptr(k_cache),
+                   _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), hkv, d, bs, nb,
+                   _stream(stream)), prepare)
 
 
 def decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int,

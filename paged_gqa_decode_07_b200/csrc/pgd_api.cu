@@ -583,7 +583,7 @@ pgd_status pgd_merge_partials(const float *o_part, const float *lse_part, int32_
     if (head_dim != 128 && head_dim != 256) return PGD_ERR_UNSUPPORTED;
     if (rows == 0) return PGD_OK;
     if (!o_part || !lse_part || !out) return PGD_ERR_INVALID_ARG;
-    if (!aligned(o_part, 4) || !aligned(lse_part, 4) || !aligned(out, 2) ||
+    if (!aligned(o_part, 16) || !aligned(lse_part, 4) || !aligned(out, 8) ||
         (lse_out && !aligned(lse_out, 4)))
         return PGD_ERR_INVALID_ARG;
     cudaError_t e = launch_merge_partials(o_part, lse_part, num_parts, rows, head_dim,

@@ -63,16 +63,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Limits of the bounded waits.  Pipeline waits (a stage, a descriptor, an
 // appended row) give up after DecodeParams::wait_ns, 1 s unless a test
 // shortens it; the producer's final drain of its own copies always allows
-// kDrainWaitNs, because every copy it issued must land before the CTA exits.
+// kDrainWaitNs (1 s), because every copy it issued must land before the CTA
+// exits.
 constexpr uint64_t kDefaultWaitNs = 1000000000ull;
-constexpr uint64_t kDrainWaitNs = 200000000ull;
+constexpr uint64_t kDrainWaitNs = kDefaultWaitNs;
+
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
 
 // Wait for the phase with the given parity to complete, for at most
 // `limit_ns` nanoseconds.  Returns false if the limit passed; the caller
 // raises the timeout flag, keeps its control flow uniform and bails out at
-// the next point where the whole CTA can agree.
+// the next point where the whole CTA can agree.  A try_wait may suspend the
+// thread for a while by itself, so a limit shortened below the default (the
+// timeout test hook) polls with the non-blocking test_wait instead, and a
+// limit of a few ns then really runs out.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   uint64_t limit_ns) {
+    if (limit_ns < kDefaultWaitNs) {
+        const uint64_t t0 = globaltimer_ns();
+        for (;;) {
+            if (mbar_test_wait(bar, parity)) return true;
+            if (globaltimer_ns() - t0 > limit_ns) return false;
+        }
+    }
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {

@@ -151,6 +151,9 @@ def test_merge_host_validation(lib):
     assert lib.pgd_merge_partials(A, A, 0, 4, 128, A, None, None) == INVALID
     assert lib.pgd_merge_partials(A, A, 2, 4, 100, A, None, None) == UNSUPPORTED
     assert lib.pgd_merge_partials(A, A, 2, 0, 128, A, None, None) == OK
+    # the merge reads float4 columns and writes 8-byte groups
+    assert lib.pgd_merge_partials(MIS, A, 2, 4, 128, A, None, None) == INVALID
+    assert lib.pgd_merge_partials(A, A, 2, 4, 128, MIS, None, None) == INVALID
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
