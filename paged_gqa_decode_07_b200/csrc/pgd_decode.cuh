@@ -680,11 +680,30 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             const int32_t *bt = p.block_table + (long long)c.s * p.max_blocks_per_seq;
             return j0 + lane < j1 ? __ldg(bt + j0 + lane) : 0;
         };
+        // The units of one sequence (its KV heads) share its block-table row,
+        // so a unit whose segment starts at the same block reuses the ids the
+        // previous unit loaded, and the next sequence's ids are loaded as soon
+        // as the walk enters a sequence: a whole sequence of units ahead.  A
+        // walk of many short units then never waits on a block-table load.
+        Cursor la = cur;             // first unit of the sequence after cur's
+        int pf_la = 0, la_j0 = -1;
+        auto look_ahead = [&](const Cursor &from) {
+            la = from;
+            while (la.a < u1 && la.s == from.s) next_unit<BS>(la, p);
+            la_j0 = -1;
+            if (la.a < u1) {
+                int b0, b1;
+                seg_of(la, b0, b1);
+                pf_la = first_ids(la, b0, b1);
+                la_j0 = b0;
+            }
+        };
         int pf = 0;
         if (cur.a < u1) {
             int a0, a1;
             seg_of(cur, a0, a1);
             pf = first_ids(cur, a0, a1);
+            look_ahead(cur);
         }
         for (; cur.a < u1 && ok;) {
             int j0, j1;                                  // absolute blocks
@@ -695,7 +714,15 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             if (nxt.a < u1) {
                 int b0, b1;
                 seg_of(nxt, b0, b1);
-                pf_next = first_ids(nxt, b0, b1);
+                if (nxt.s == cur.s && b0 == j0) {
+                    pf_next = pf;                        // same row, same first block
+                } else if (nxt.s == la.s && b0 == la_j0) {
+                    pf_next = pf_la;                     // loaded a sequence ago
+                    look_ahead(nxt);
+                } else {
+                    pf_next = first_ids(nxt, b0, b1);
+                    look_ahead(nxt);
+                }
             }
             if (j0 >= j1) {          // the range holds only this unit's fixed-cost slots
                 cur = nxt;
