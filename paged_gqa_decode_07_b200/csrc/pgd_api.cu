@@ -207,9 +207,6 @@ std::atomic<int> g_math{PGD_MATH_TENSOR_CORE};
 // Limit of the decode kernels' pipeline waits in ns (pgd_debug_set_wait_limit_ns).
 std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
 
-// Whole units of at most one stage of tiles go to one consumer warp each.
-constexpr int32_t kShortUnits = 1;
-
 template <int CC>
 bool pick_cuda_core(int bs, Variant *v) {
     if (bs == 16) *v = {&launch_decode<128, 16, 1, false, CC>, &decode_ctas_per_sm<128, 16, 1, false, CC>};
@@ -472,7 +469,6 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     p.rows = rows;
     p.out_f32 = out_f32 ? 1 : 0;
     p.wait_ns = g_wait_ns.load();
-    p.short_units = kShortUnits;
     a.grid = static_cast<int>(grid);
     a.stream = s;
     cudaError_t e = var.launch(a);
@@ -804,7 +800,6 @@ extern "C" pgd_status pgd_paged_decode_attention_noalloc(
     p.window = 0;
     p.rows = g;
     p.wait_ns = g_wait_ns.load();
-    p.short_units = kShortUnits;
     a.grid = static_cast<int>(grid);
     a.stream = s;
     e = var.launch(a);

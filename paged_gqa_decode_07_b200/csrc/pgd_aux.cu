@@ -55,15 +55,6 @@ cudaError_t launch_kv_append(const void *k_new, const void *v_new, const int64_t
     return cudaGetLastError();
 }
 
-// Two fp32 values -> two E4M3 bytes (round to nearest even, saturating at
-// +-448), lo in the low byte.
-__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
-    uint32_t r;
-    asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %2, %1;\n\tcvt.u32.u16 %0, t;\n\t}"
-        : "=r"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-
 // Quantising append: bf16 K/V rows of new tokens into an FP8 E4M3 cache
 // ("attention kernels", "what to check": FP8 KV).  Each element is divided by
 // its KV head's fp32 scale (IEEE division) and rounded to E4M3.  One warp per

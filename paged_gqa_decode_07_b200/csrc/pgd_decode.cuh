@@ -86,8 +86,6 @@ struct DecodeParams {
     // limit of every pipeline wait in ns (kDefaultWaitNs unless a test of
     // the timeout path shortens it)
     uint64_t wait_ns;
-    // 1: a whole unit that fits in one stage goes to one consumer warp alone
-    int32_t short_units;
 };
 
 constexpr int kConsumerWarps = 4;
@@ -100,16 +98,12 @@ constexpr float kLn2 = 0.6931471805599453f;
 // moves a row's reference max (lazy rescaling)
 constexpr float kLazyRescale = 8.f;
 constexpr uint32_t kBarConsumers = 1;
-// segment kinds (SegDesc::kind); 0 .. 3 name the one consumer warp that
-// processes a short unit alone
-constexpr int kSegTerminal = -1;   // no more segments for this CTA
-constexpr int kSegShared = 4;      // every consumer warp takes a share of the tokens
 
 // Segment descriptor written by the producer, read by the consumers.
 struct SegDesc {
     long long u;      // flattened index of the segment's first tile
     int s, h, j0, j1, n, ctx;
-    int kind;         // kSegTerminal, kSegShared, or the warp of a short unit
+    int terminal;     // 1: no more segments for this CTA
     float ksc, vsc;   // FP8 per-KV-head scales (1 for bf16)
     int jlo;          // first block any query row of the unit sees
 };
@@ -147,11 +141,6 @@ struct DecodeCfg {
     static constexpr bool QPAD = CC == 0;
     static constexpr int QROW = QPAD ? D * 2 + (FP8 ? 32 : 16) : D * 2;
     static constexpr int QSLOT = NP * QROW;              // query rows of one unit
-    // Short units (whole in the CTA, at most one stage of tiles) may go to one
-    // consumer warp each, which then needs every row of the unit in its own
-    // registers: up to 8 rows, query fragments held in registers (the 16-row
-    // variant has no registers to spare for the extra output path).
-    static constexpr bool SHORT = CC == 0 && NT == 1 && !QSMEM;
     // descriptor ring depth (one slot for 16 or more query rows at head_dim
     // 128, so that two CTAs still fit on an SM; one for 32 rows at 256)
     static constexpr int NSEG =
@@ -660,7 +649,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         Cursor cur = first_unit<BS>(p, misc->s0, misc->pfx0, u0, win0);
         const uint32_t qtok = (uint32_t)(g * D * 2);          // one query token's rows
         uint32_t it = 0, sit = 0, ait = 0;
-        uint32_t nshort = 0;                                  // short units so far
         bool ok = true;
         // FP8 scales of the first 32 KV heads, one per lane
         float ks_l = 1.f, vs_l = 1.f;
@@ -739,13 +727,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     vsc = __ldg(p.v_scale + cur.h);
                 }
             }
-            // A whole unit whose tiles fit in one stage goes to one consumer
-            // warp alone, round robin over the CTA's short units: the four
-            // warps then work on four units at once, and none of them waits
-            // for a merge across warps.
-            int kind = kSegShared;
-            if (C::SHORT && p.short_units && j0 == cur.jlo && j1 == cur.n && j1 - j0 <= C::BPS)
-                kind = (int)(nshort++ & 3u);
             // -- descriptor and query rows of the segment
             {
                 const uint32_t slot = sit % C::NSEG;
@@ -762,7 +743,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     d.j1 = j1;
                     d.n = cur.n;
                     d.ctx = cur.ctx;
-                    d.kind = kind;
+                    d.terminal = 0;
                     d.ksc = ksc;
                     d.vsc = vsc;
                     d.jlo = cur.jlo;
@@ -861,7 +842,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     raise_flag(p.flags, kFlagTimeout);
             // terminal descriptor (also after a timeout, so that the consumers stop)
             if (free_slot) {
-                segs[slot].kind = kSegTerminal;
+                segs[slot].terminal = 1;
                 mbar_arrive(seg_full + 8 * slot);
             }
         }
@@ -885,17 +866,13 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         const int j1 = (int)lds32(da + offsetof(SegDesc, j1));
         const int nunit = (int)lds32(da + offsetof(SegDesc, n));
         const int ctx = (int)lds32(da + offsetof(SegDesc, ctx));
-        const int kind = (int)lds32(da + offsetof(SegDesc, kind));
+        const int terminal = (int)lds32(da + offsetof(SegDesc, terminal));
         const float ksc = __uint_as_float(lds32(da + offsetof(SegDesc, ksc)));
         const float vsc = __uint_as_float(lds32(da + offsetof(SegDesc, vsc)));
         const int jlo = (int)lds32(da + offsetof(SegDesc, jlo));
-        // A short unit belongs to one warp and needs no barrier.  Every other
-        // segment (and a wait that timed out, whose descriptor may be stale)
-        // meets all consumer warps at a barrier that also agrees on leaving.
-        const bool alone = C::SHORT && seg_ok && kind >= 0 && kind < kSegShared;
-        if (!alone &&
-            named_bar_sync_or(kBarConsumers, kConsumers, !seg_ok || kind == kSegTerminal))
-            return;
+        // all consumers agree on leaving (a terminal descriptor, or a wait that
+        // timed out, whose descriptor may be stale)
+        if (named_bar_sync_or(kBarConsumers, kConsumers, !seg_ok || terminal)) return;
         const bool whole = (j0 == jlo && j1 == nunit);
         const int R = p.rows;
 
@@ -954,25 +931,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         };
 
         if constexpr (CC == 0) {
-            if (alone && warp != kind) {
-                // another warp's short unit: free the descriptor slot, and its
-                // one stage once it has landed (so that this warp's arrivals
-                // stay in step with the ring's phases)
-                __syncwarp();
-                if (lane == 0) mbar_arrive(seg_empty + 8 * qs);
-                ++sit;
-                const uint32_t slot = it % NSTAGES;
-                const bool ok = mbar_wait_bounded(bar_full + 8 * slot, (it / NSTAGES) & 1, p.wait_ns);
-                ++it;
-                if (!ok) {
-                    raise_flag(p.flags, kFlagTimeout);
-                    named_bar_sync_or(kBarConsumers, kConsumers, true);   // leave with the others
-                    return;
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_empty + 8 * slot);
-                continue;
-            }
             // This warp's row group: rows rbase .. rbase + 8 * NTW - 1 (all rows
             // unless the unit has 32, when warps 0, 1 take rows 0-15 and warps 2,
             // 3 rows 16-31)
@@ -1020,12 +978,16 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     }
                 }
                 if constexpr (FP8) {
-                    // The FP8 product runs in f16, whose range is narrower than
-                    // bf16's.  The unit's query rows are scaled by a power of two
-                    // 2^sh that puts their largest magnitude in [2^14, 2^15), so no
-                    // value overflows and small ones keep their bits, and the
-                    // score scale takes 2^-sh back (both exact).  The warps of a
-                    // row group read the same rows, so they pick the same sh.
+                    // The FP8 scores run on the E4M3 tensor-core product (K straight
+                    // from the cache bytes, no conversion).  The unit's query rows
+                    // are scaled by the power of two 2^sh that puts their largest
+                    // magnitude in [128, 256) (the score scale takes 2^-sh back,
+                    // exactly), and each value x is carried as two E4M3 terms, hi =
+                    // E4M3(x) and lo = E4M3(x - hi), about 7 significant bits in
+                    // all.  The warps of a row group read the same rows, so they
+                    // pick the same sh.  Register k holds d = 16k + 4t .. 16k + 4t + 3
+                    // (hi in [0], lo in [1]): k = 2kk, 2kk + 1 are the B operand of
+                    // k-step kk.
                     float qmax = 0.f;
 #pragma unroll
                     for (int k = 0; k < C::KSTEPS; ++k)
@@ -1039,19 +1001,26 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
 #pragma unroll
                     for (int off = 16; off; off >>= 1)
                         qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, off));
-                    const int ex = qmax > 0.f ? (int)((__float_as_uint(qmax) >> 23) & 0xffu) - 127 : 14;
-                    const int sh = min(100, max(-100, 14 - ex));
+                    const int ex = qmax > 0.f ? (int)((__float_as_uint(qmax) >> 23) & 0xffu) - 127 : 7;
+                    const int sh = min(100, max(-100, 7 - ex));
                     const float up = __uint_as_float((uint32_t)(127 + sh) << 23);
                     sl2 *= __uint_as_float((uint32_t)(127 - sh) << 23);
 #pragma unroll
                     for (int k = 0; k < C::KSTEPS; ++k)
 #pragma unroll
-                        for (int nt = 0; nt < C::NTW; ++nt)
-#pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const float2 f = unpack_bf16x2(qf[k][nt][e]);
-                                qf[k][nt][e] = pack_f16x2(f.x * up, f.y * up);
-                            }
+                        for (int nt = 0; nt < C::NTW; ++nt) {
+                            const float2 f0 = unpack_bf16x2(qf[k][nt][0]);
+                            const float2 f1 = unpack_bf16x2(qf[k][nt][1]);
+                            const float x[4] = {f0.x * up, f0.y * up, f1.x * up, f1.y * up};
+                            const uint32_t h01 = f32x2_to_e4m3x2(x[0], x[1]);
+                            const uint32_t h23 = f32x2_to_e4m3x2(x[2], x[3]);
+                            const float2 g0 = unpack_f16x2(e4m3x2_to_f16x2(h01));
+                            const float2 g1 = unpack_f16x2(e4m3x2_to_f16x2(h23));
+                            const uint32_t l01 = f32x2_to_e4m3x2(x[0] - g0.x, x[1] - g0.y);
+                            const uint32_t l23 = f32x2_to_e4m3x2(x[2] - g1.x, x[3] - g1.y);
+                            qf[k][nt][0] = h01 | (h23 << 16);
+                            qf[k][nt][1] = l01 | (l23 << 16);
+                        }
                 }
             }
             if (!C::QSMEM) {
@@ -1093,13 +1062,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 }
                 const uint32_t sK = sbase + slot * C::STAGE, sV = sK + C::STAGE_KV;
 
-                // 16-token sub-tiles of this warp: its own 16 (or 32) tokens of
-                // the stage, or every token of a short unit it holds alone
-                const int nsub = alone ? (n_valid + 15) / 16 : C::SUBS;
-                for (int sub = 0; sub < nsub; ++sub) {
+                // this warp's 16-token sub-tiles: its own 16 (or 32) tokens of the stage
+                for (int sub = 0; sub < C::SUBS; ++sub) {
                     // first stage token of this warp's 16-token sub-tile
-                    const int tb = alone ? 16 * sub
-                                         : (C::RG == 1 ? 16 * warp : 32 * (warp & 1) + 16 * sub);
+                    const int tb = C::RG == 1 ? 16 * warp : 32 * (warp & 1) + 16 * sub;
                     if (tb < n_valid) {
                         // ---- S^T = K . Q^T for this warp's 16 tokens (two MMA chains)
                         float sacc[C::NTW][4], sac2[C::NTW][4];
@@ -1145,22 +1111,22 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                 }
                             }
                         } else {
+                            // A fragments: 4 consecutive d of tokens tb + gid and tb + gid
+                            // + 8, from 16-byte chunks 2kk and 2kk + 1 of each row
                             const int tok0 = tb + gid, tok1 = tok0 + 8;
                             const int r0 = tok0 % BS, r1 = tok1 % BS;
                             const uint32_t base0 = sK + (tok0 / BS) * C::TILE + r0 * 128 + 4 * t4;
                             const uint32_t base1 = sK + (tok1 / BS) * C::TILE + r1 * 128 + 4 * t4;
 #pragma unroll
-                            for (int k = 0; k < C::KSTEPS; ++k) {
-                                const uint32_t w0 = lds32(base0 + ((k ^ (r0 & 7)) << 4));
-                                const uint32_t w1 = lds32(base1 + ((k ^ (r1 & 7)) << 4));
-                                const uint32_t a0 = e4m3x2_to_f16x2(w0 & 0xffffu);
-                                const uint32_t a2 = e4m3x2_to_f16x2(w0 >> 16);
-                                const uint32_t a1 = e4m3x2_to_f16x2(w1 & 0xffffu);
-                                const uint32_t a3 = e4m3x2_to_f16x2(w1 >> 16);
+                            for (int kk = 0; kk < C::KSTEPS / 2; ++kk) {
+                                const uint32_t a0 = lds32(base0 + (((2 * kk) ^ (r0 & 7)) << 4));
+                                const uint32_t a1 = lds32(base1 + (((2 * kk) ^ (r1 & 7)) << 4));
+                                const uint32_t a2 = lds32(base0 + (((2 * kk + 1) ^ (r0 & 7)) << 4));
+                                const uint32_t a3 = lds32(base1 + (((2 * kk + 1) ^ (r1 & 7)) << 4));
 #pragma unroll
                                 for (int nt = 0; nt < C::NTW; ++nt) {
-                                    if (k & 1) mma_f16(sac2[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
-                                    else       mma_f16(sacc[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
+                                    mma_e4m3(sacc[nt], a0, a1, a2, a3, qf[2 * kk][nt][0], qf[2 * kk + 1][nt][0]);
+                                    mma_e4m3(sac2[nt], a0, a1, a2, a3, qf[2 * kk][nt][1], qf[2 * kk + 1][nt][1]);
                                 }
                             }
                         }
@@ -1338,73 +1304,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 if (!FP8) return 16 * mt + gid + (e >> 1) * 8;
                 return 16 * gid + 2 * mt + (e >> 1);
             };
-            if (alone) {
-                // The warp holds the short unit's whole softmax state: out (or the
-                // fp32 result) and lse go straight from its accumulators.
-                if (abort) {
-                    named_bar_sync_or(kBarConsumers, kConsumers, true);   // leave with the others
-                    return;
-                }
-                float inv[C::NTW][2];
-#pragma unroll
-                for (int nt = 0; nt < C::NTW; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        float l = l_run[nt][e];
-#pragma unroll
-                        for (int off = 4; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-                        inv[nt][e] = l > 0.f ? vsc / l : 0.f;
-                        const int r = nt * 8 + 2 * t4 + e;
-                        if (p.lse_out && gid == 0 && r < R)
-                            p.lse_out[orow(r)] = l > 0.f ? (m_run[nt][e] + log2f(l)) * kLn2 : -INFINITY;
-                    }
-                if (p.out_f32) {
-                    float *of = reinterpret_cast<float *>(p.out);
-#pragma unroll
-                    for (int mt = 0; mt < C::DT; ++mt)
-#pragma unroll
-                        for (int nt = 0; nt < C::NTW; ++nt)
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int r = nt * 8 + 2 * t4 + (e & 1);
-                                if (r < R) of[orow(r) * D + dim_of(mt, e)] = o[mt][nt][e] * inv[nt][e & 1];
-                            }
-                } else if constexpr (!FP8) {
-                    // a warp transpose of each 8x8 half gives lane (gid, t4) query
-                    // row 8nt + gid at dims 16mt + 8hf + 2t4 and the next one
-#pragma unroll
-                    for (int mt = 0; mt < C::DT; ++mt)
-#pragma unroll
-                        for (int nt = 0; nt < C::NTW; ++nt)
-#pragma unroll
-                            for (int hf = 0; hf < 2; ++hf) {
-                                const uint32_t t = movmatrix_trans(
-                                    pack_bf16x2(o[mt][nt][2 * hf] * inv[nt][0],
-                                                o[mt][nt][2 * hf + 1] * inv[nt][1]));
-                                const int r = nt * 8 + gid;
-                                if (r < R)
-                                    *reinterpret_cast<uint32_t *>(p.out + orow(r) * D + 16 * mt +
-                                                                  8 * hf + 2 * t4) = t;
-                            }
-                } else {
-                    // FP8 layout: elements c and c + 2 are dims 16gid + 2mt and the
-                    // next one of query row 8nt + 2t4 + c
-#pragma unroll
-                    for (int mt = 0; mt < C::DT; ++mt)
-#pragma unroll
-                        for (int nt = 0; nt < C::NTW; ++nt)
-#pragma unroll
-                            for (int c = 0; c < 2; ++c) {
-                                const int r = nt * 8 + 2 * t4 + c;
-                                if (r < R)
-                                    *reinterpret_cast<uint32_t *>(p.out + orow(r) * D + 16 * gid +
-                                                                  2 * mt) =
-                                        pack_bf16x2(o[mt][nt][c] * inv[nt][c],
-                                                    o[mt][nt][c + 2] * inv[nt][c]);
-                            }
-                }
-                continue;
-            }
             // A: warps 0, 1; B: warps 2, 3
             auto store_rows = [&](int nt) {
                 float *buf = reinterpret_cast<float *>(

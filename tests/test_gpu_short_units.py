@@ -1,12 +1,12 @@
-"""GPU parity of the short-unit path: a (sequence, KV head) unit that lies
-whole in one CTA's range and fits in one 64-token stage is processed by one
-consumer warp alone, which writes out and lse from its own accumulators.
-Batches made mostly of such units (the continuous-batching mix of the
-"attention kernels" page, section "paged KV and kernels": many short
-sequences next to a few long ones, in one launch) are compared with the
-oracle row by row, in every output form the path writes: bf16 out and lse,
-the fp32 split result of pgd_paged_decode_partial, several query tokens, a
-window, the fused append, and both KV formats."""
+"""GPU parity on batches made mostly of short (sequence, KV head) units:
+many units that lie whole in one CTA's range and fit in one 64-token stage,
+next to a few long ones (the continuous-batching mix of the "attention
+kernels" page, section "paged KV and kernels": short and long sequences in
+one launch).  The batches are compared with the oracle row by row in every
+output form: bf16 out and lse, the fp32 split result of
+pgd_paged_decode_partial, several query tokens, a window, the fused append,
+and both KV formats; the short units' results must also be identical across
+repeated runs and grids of every size."""
 import numpy as np
 import pytest
 import torch
@@ -54,8 +54,8 @@ def test_many_short_units(Hq, Hkv, bs, dt):
 
 @pytest.mark.parametrize("num_ctas", [1, 5, 64, 296, 1000])
 def test_short_units_any_grid(num_ctas):
-    """The cut decides which units are whole in a CTA (short path) and which
-    are split (shared path and merge): every grid must give the oracle's
+    """The cut decides which units are whole in a CTA and which are split
+    (pieces merged by log-sum-exp): every grid must give the oracle's
     result."""
     w = make_case(short_mix(200, 1110, longest=80, long_ones=(5000, 700)), 64, 8, 128, 16,
                   "e4m3", seed=1111, name="short-grid")
@@ -95,8 +95,8 @@ def test_short_units_multi_token_and_window(L, W):
 
 @pytest.mark.parametrize("dt", ["bf16", "e4m3"])
 def test_short_units_fp32_split_result(dt):
-    """pgd_paged_decode_partial writes the unrounded fp32 result, which the
-    short path stores element by element."""
+    """pgd_paged_decode_partial writes the unrounded fp32 result of every
+    short unit."""
     w = make_case(short_mix(120, 1140), 32, 8, 128, 16, dt, seed=1141, name="short-f32")
     d = Dev(w)
     o, lse = pgd.paged_decode_partial(d.q, d.k, d.v, d.bt, d.cl, 32, 8, 128, 16, w.scale,
