@@ -145,12 +145,13 @@ struct WsLayout {
     size_t lse, opart, total;
 };
 
-// Caller or library workspace: split partials only (no zeroing needed).
-WsLayout ws_layout(int g, int D, long long grid) {
+// Caller or library workspace: split partials only (no zeroing needed), two
+// slots of g rows per range, `ranges` ranges.
+WsLayout ws_layout(int g, int D, long long ranges) {
     WsLayout w;
     w.lse = 0;
-    w.opart = round256(sizeof(float) * 2 * grid * g);
-    w.total = w.opart + round256(sizeof(float) * 2 * grid * g * D);
+    w.opart = round256(sizeof(float) * 2 * ranges * g);
+    w.total = w.opart + round256(sizeof(float) * 2 * ranges * g * D);
     return w;
 }
 
@@ -339,7 +340,7 @@ size_t pgd_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t
     DeviceState *d = nullptr;
     if (device_state(&d) != PGD_OK) return 0;
     const long long grid = static_cast<long long>(d->sms) * kMaxCtasPerSmForSizing;
-    return ws_layout(num_q_heads / num_kv_heads, head_dim, grid).total;
+    return ws_layout(num_q_heads / num_kv_heads, head_dim, grid * kRangesPerShare).total;
 }
 
 }  // extern "C"
@@ -407,10 +408,13 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     if (grid > (1LL << 24)) return PGD_ERR_INVALID_ARG;
 
     // ---- workspace --------------------------------------------------------------
-    const WsLayout lay = ws_layout(rows, head_dim, grid);
+    // a CTA's share may be cut into its main part and kTailChunks chunks
+    const WsLayout lay = ws_layout(rows, head_dim, grid * kRangesPerShare);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if ((st = ensure_counters(d, static_cast<long long>(num_seqs) * num_kv_heads, s)) != PGD_OK)
+    // arrival counters per unit, then a claim counter per CTA and a done count
+    if ((st = ensure_counters(d, static_cast<long long>(num_seqs) * num_kv_heads + grid + 1, s)) !=
+        PGD_OK)
         return st;
     if (!ws) {
         std::lock_guard<std::mutex> lk(g_mu);
@@ -469,6 +473,7 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     p.rows = rows;
     p.out_f32 = out_f32 ? 1 : 0;
     p.wait_ns = g_wait_ns.load();
+    p.tails_ok = 1;
     a.grid = static_cast<int>(grid);
     a.stream = s;
     cudaError_t e = var.launch(a);
@@ -800,6 +805,7 @@ extern "C" pgd_status pgd_paged_decode_attention_noalloc(
     p.window = 0;
     p.rows = g;
     p.wait_ns = g_wait_ns.load();
+    p.tails_ok = 0;   // the static array holds one range per CTA and no claim counters
     a.grid = static_cast<int>(grid);
     a.stream = s;
     e = var.launch(a);
