@@ -705,13 +705,11 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         // appender warp writes the appended rows; in a chunk the producer does.
         long long rs = u0, re = u1m;
         bool in_main = true;
-        // the segment's blocks [j0, j1) of unit c in range [a, b) (empty: only
-        // fixed-cost slots)
-        auto seg_in = [&](const Cursor &c, long long a, long long b, int &j0, int &j1) {
-            j0 = c.jlo + (int)max(0LL, a - c.a);
-            j1 = c.jlo + (int)min((long long)(c.n - c.jlo), b - c.a);
+        // the segment's blocks [j0, j1) of unit c (empty: only fixed-cost slots)
+        auto seg_of = [&](const Cursor &c, int &j0, int &j1) {
+            j0 = c.jlo + (int)max(0LL, rs - c.a);
+            j1 = c.jlo + (int)min((long long)(c.n - c.jlo), re - c.a);
         };
-        auto seg_of = [&](const Cursor &c, int &j0, int &j1) { seg_in(c, rs, re, j0, j1); };
         // block ids of a segment's first 32 blocks, one per lane; the next
         // unit's are loaded while this unit's tiles are issued, so the walk
         // never waits on a dependent block-table load
@@ -746,58 +744,21 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 look_ahead(cur);
             }
         };
-        // move cursor c forward to the unit that holds work index x (whole
+        // move cur forward to the unit that holds work index x (whole
         // sequences at a time, then heads)
-        auto seek = [&](Cursor &c, long long x) {
-            while (c.a + (long long)(Hkv - c.h) * c.w <= x) {
-                c.a += (long long)(Hkv - 1 - c.h) * c.w;
-                c.h = Hkv - 1;
-                next_unit<BS>(c, p);
+        auto seek = [&](long long x) {
+            while (cur.a + (long long)(Hkv - cur.h) * cur.w <= x) {
+                cur.a += (long long)(Hkv - 1 - cur.h) * cur.w;
+                cur.h = Hkv - 1;
+                next_unit<BS>(cur, p);
             }
-            const long long hs = (x - c.a) / c.w;
-            c.h += (int)hs;
-            c.a += hs * c.w;
+            const long long hs = (x - cur.a) / cur.w;
+            cur.h += (int)hs;
+            cur.a += hs * cur.w;
         };
-        // Claims run one range ahead: the claim for the range after the
-        // current one is issued when the current one starts, and read (with
-        // the block ids of the claimed chunk's first unit loaded) when the
-        // walk reaches the current range's last unit, so a range change costs
-        // the walk no round trip.  The CTA whose tail chunks are claimed next:
-        // its own first, then the shares to its right.
+        // the CTA whose tail chunks are claimed next: own first, then to the right
         long long claim_share = cta;
         int *const claims = p.counters + (long long)B * Hkv;   // [G] claims, [gridDim.x] done
-        int pend = 0;              // result of the claim in flight (lane 0)
-        bool pend_live = false;
-        long long next_range = -1; // the range after the current one, once resolved
-        Cursor ncur = cur;         // its first unit
-        int npf = 0;               // and that unit's first block ids
-        auto issue_claim = [&]() {
-            pend_live = false;
-            if (rg.tails && claim_share < G && claim_share <= cta + kStealReach) {
-                if (lane == 0) pend = atomicAdd(claims + claim_share, 1);
-                pend_live = true;
-            }
-        };
-        auto resolve_next = [&](const Cursor &from) {
-            next_range = -1;
-            while (pend_live) {
-                const int i = __shfl_sync(0xffffffffu, pend, 0);
-                if (i < kTailChunks) {
-                    next_range = claim_share * kRangesPerShare + 1 + i;
-                    break;
-                }
-                ++claim_share;                           // that share's tail is taken
-                issue_claim();
-            }
-            if (next_range >= 0) {
-                const long long a = rg.start(next_range), b = rg.start(next_range + 1);
-                ncur = from;                             // from.a <= a: walk forward
-                seek(ncur, a);
-                int b0, b1;
-                seg_in(ncur, a, b, b0, b1);
-                npf = first_ids(ncur, b0, b1);
-            }
-        };
         // the producer writes the appended row of a tail-chunk unit itself
         auto append_row = [&](const Cursor &c) {
             int pb = __ldg(p.block_table + (long long)c.s * p.max_blocks_per_seq + c.n - 1);
@@ -819,9 +780,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             __syncwarp();
         };
         enter_range();
-        issue_claim();
         for (;;) {                                       // ranges
-        bool resolved = false;
         Cursor last = cur;                               // the last unit walked
         for (; cur.a < re && ok;) {
             int j0, j1;                                  // absolute blocks
@@ -841,9 +800,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     pf_next = first_ids(nxt, b0, b1);
                     look_ahead(nxt);
                 }
-            } else if (!resolved) {                      // the range's last unit
-                resolve_next(cur);
-                resolved = true;
             }
             last = cur;
             if (j0 >= j1) {          // the range holds only this unit's fixed-cost slots
@@ -953,15 +909,25 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             pf = pf_next;
         }
         if (!ok || !rg.tails) break;
-        if (!resolved) resolve_next(last);
-        if (next_range < 0) break;
-        rs = rg.start(next_range);
-        re = rg.start(next_range + 1);
+        // claim the next tail chunk: this CTA's own first, then its neighbours'
+        long long chunk = -1;
+        while (claim_share < G && claim_share <= cta + kStealReach) {
+            int i = 0;
+            if (lane == 0) i = atomicAdd(claims + claim_share, 1);
+            i = __shfl_sync(0xffffffffu, i, 0);
+            if (i < kTailChunks) {
+                chunk = claim_share * kRangesPerShare + 1 + i;
+                break;
+            }
+            ++claim_share;
+        }
+        if (chunk < 0) break;
+        rs = rg.start(chunk);
+        re = rg.start(chunk + 1);
         in_main = false;
-        cur = ncur;
-        pf = npf;
-        look_ahead(cur);
-        issue_claim();
+        cur = last;                                      // cur.a <= rs: walk forward
+        seek(rs);
+        enter_range();
         }                                                // ranges
         if (rg.tails && ok) {
             // this CTA has made its last claim; the last CTA to get here resets
