@@ -1104,16 +1104,13 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     }
                 }
                 if constexpr (FP8) {
-                    // The FP8 scores run on the E4M3 tensor-core product (K straight
-                    // from the cache bytes, no conversion).  The unit's query rows
-                    // are scaled by the power of two 2^sh that puts their largest
-                    // magnitude in [128, 256) (the score scale takes 2^-sh back,
-                    // exactly), and each value x is carried as two E4M3 terms, hi =
-                    // E4M3(x) and lo = E4M3(x - hi), about 7 significant bits in
-                    // all.  The warps of a row group read the same rows, so they
-                    // pick the same sh.  Register k holds d = 16k + 4t .. 16k + 4t + 3
-                    // (hi in [0], lo in [1]): k = 2kk, 2kk + 1 are the B operand of
-                    // k-step kk.
+                    // The FP8 product runs in f16 (every E4M3 value is an f16
+                    // value), whose range is narrower than bf16's.  The unit's
+                    // query rows are scaled by a power of two 2^sh that puts their
+                    // largest magnitude in [2^14, 2^15), so no value overflows and
+                    // small ones keep their bits, and the score scale takes 2^-sh
+                    // back (both exact).  The warps of a row group read the same
+                    // rows, so they pick the same sh.
                     float qmax = 0.f;
 #pragma unroll
                     for (int k = 0; k < C::KSTEPS; ++k)
@@ -1127,26 +1124,19 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
 #pragma unroll
                     for (int off = 16; off; off >>= 1)
                         qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, off));
-                    const int ex = qmax > 0.f ? (int)((__float_as_uint(qmax) >> 23) & 0xffu) - 127 : 7;
-                    const int sh = min(100, max(-100, 7 - ex));
+                    const int ex = qmax > 0.f ? (int)((__float_as_uint(qmax) >> 23) & 0xffu) - 127 : 14;
+                    const int sh = min(100, max(-100, 14 - ex));
                     const float up = __uint_as_float((uint32_t)(127 + sh) << 23);
                     sl2 *= __uint_as_float((uint32_t)(127 - sh) << 23);
 #pragma unroll
                     for (int k = 0; k < C::KSTEPS; ++k)
 #pragma unroll
-                        for (int nt = 0; nt < C::NTW; ++nt) {
-                            const float2 f0 = unpack_bf16x2(qf[k][nt][0]);
-                            const float2 f1 = unpack_bf16x2(qf[k][nt][1]);
-                            const float x[4] = {f0.x * up, f0.y * up, f1.x * up, f1.y * up};
-                            const uint32_t h01 = f32x2_to_e4m3x2(x[0], x[1]);
-                            const uint32_t h23 = f32x2_to_e4m3x2(x[2], x[3]);
-                            const float2 g0 = unpack_f16x2(e4m3x2_to_f16x2(h01));
-                            const float2 g1 = unpack_f16x2(e4m3x2_to_f16x2(h23));
-                            const uint32_t l01 = f32x2_to_e4m3x2(x[0] - g0.x, x[1] - g0.y);
-                            const uint32_t l23 = f32x2_to_e4m3x2(x[2] - g1.x, x[3] - g1.y);
-                            qf[k][nt][0] = h01 | (h23 << 16);
-                            qf[k][nt][1] = l01 | (l23 << 16);
-                        }
+                        for (int nt = 0; nt < C::NTW; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const float2 f = unpack_bf16x2(qf[k][nt][e]);
+                                qf[k][nt][e] = pack_f16x2(f.x * up, f.y * up);
+                            }
                 }
             }
             if (!C::QSMEM) {
@@ -1237,22 +1227,22 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                 }
                             }
                         } else {
-                            // A fragments: 4 consecutive d of tokens tb + gid and tb + gid
-                            // + 8, from 16-byte chunks 2kk and 2kk + 1 of each row
                             const int tok0 = tb + gid, tok1 = tok0 + 8;
                             const int r0 = tok0 % BS, r1 = tok1 % BS;
                             const uint32_t base0 = sK + (tok0 / BS) * C::TILE + r0 * 128 + 4 * t4;
                             const uint32_t base1 = sK + (tok1 / BS) * C::TILE + r1 * 128 + 4 * t4;
 #pragma unroll
-                            for (int kk = 0; kk < C::KSTEPS / 2; ++kk) {
-                                const uint32_t a0 = lds32(base0 + (((2 * kk) ^ (r0 & 7)) << 4));
-                                const uint32_t a1 = lds32(base1 + (((2 * kk) ^ (r1 & 7)) << 4));
-                                const uint32_t a2 = lds32(base0 + (((2 * kk + 1) ^ (r0 & 7)) << 4));
-                                const uint32_t a3 = lds32(base1 + (((2 * kk + 1) ^ (r1 & 7)) << 4));
+                            for (int k = 0; k < C::KSTEPS; ++k) {
+                                const uint32_t w0 = lds32(base0 + ((k ^ (r0 & 7)) << 4));
+                                const uint32_t w1 = lds32(base1 + ((k ^ (r1 & 7)) << 4));
+                                const uint32_t a0 = e4m3x2_to_f16x2(w0 & 0xffffu);
+                                const uint32_t a2 = e4m3x2_to_f16x2(w0 >> 16);
+                                const uint32_t a1 = e4m3x2_to_f16x2(w1 & 0xffffu);
+                                const uint32_t a3 = e4m3x2_to_f16x2(w1 >> 16);
 #pragma unroll
                                 for (int nt = 0; nt < C::NTW; ++nt) {
-                                    mma_e4m3(sacc[nt], a0, a1, a2, a3, qf[2 * kk][nt][0], qf[2 * kk + 1][nt][0]);
-                                    mma_e4m3(sac2[nt], a0, a1, a2, a3, qf[2 * kk][nt][1], qf[2 * kk + 1][nt][1]);
+                                    if (k & 1) mma_f16(sac2[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
+                                    else       mma_f16(sacc[nt], a0, a1, a2, a3, qf[k][nt][0], qf[k][nt][1]);
                                 }
                             }
                         }
