@@ -160,14 +160,10 @@ size_t pgd_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
  * tiles through a TMA shared-memory pipeline, reads each K/V tile once for
  * all g query heads of its group, and keeps an online softmax; a sequence
  * whose tiles fall into several CTAs is merged by log-sum-exp by the CTA that
- * finishes its last share ("prefill and decode attention").  When there is
- * enough work, the last eighth of every share is cut into chunks that a CTA
- * which has finished its own work claims (its own first, then its
- * neighbours'), so CTAs on slower SMs do not set the step time; the cut is
- * fixed, so the chunks' results and their merge do not depend on who claims
- * them.  The result does not depend on where the blocks sit in the pool, and
- * repeated calls with the same inputs and grid give the same bits (the
- * splits are merged in a fixed order).
+ * finishes its last share ("prefill and decode attention").  The result does
+ * not depend on where the blocks sit in the pool, and repeated calls with the
+ * same inputs and grid give the same bits (the splits are merged in a fixed
+ * order).
  *
  *   q             device bf16 [num_seqs][num_q_heads][head_dim], 16-byte aligned
  *   k_cache, v_cache  device, HND layout, 16-byte aligned, num_blocks blocks
@@ -191,9 +187,8 @@ size_t pgd_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
  *                 least pgd_decode_workspace_bytes(...) bytes (any contents);
  *                 NULL/0 selects a library-owned buffer (grown on demand with
  *                 cudaMalloc, kept until pgd_shutdown()).  The library also
- *                 keeps one int32 arrival counter per (sequence, KV head) and
- *                 one claim counter per CTA in its own zeroed device buffer
- *                 (grown the same way).  Calls
+ *                 keeps one int32 arrival counter per (sequence, KV head) in
+ *                 its own zeroed device buffer (grown the same way).  Calls
  *                 that share a workspace, or run on one device at the same
  *                 time, must not overlap on the GPU.
  *   num_ctas      0 = automatic grid: one wave of resident CTAs (SM count x
@@ -443,10 +438,7 @@ pgd_status pgd_merge_partials(const float *o_part, const float *lse_part,
  * flags raised by earlier calls on this device.  Returns PGD_OK when none
  * was raised, PGD_ERR_DEVICE_BOUNDS or PGD_ERR_TIMEOUT otherwise (and
  * *flags, if non-NULL, receives the raw bit set: 1 block id, 2 context
- * length, 4 slot, 8 wait timeout).  When a flag was raised it also re-zeroes
- * the library's arrival and claim counters, which a launch that bailed out
- * may have left behind: after a flagged call, call this before the next
- * decode on the device.
+ * length, 4 slot, 8 wait timeout).
  */
 pgd_status pgd_get_device_error(void *stream, uint32_t *flags);
 

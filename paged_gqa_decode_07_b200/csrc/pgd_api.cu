@@ -145,13 +145,12 @@ struct WsLayout {
     size_t lse, opart, total;
 };
 
-// Caller or library workspace: split partials only (no zeroing needed), two
-// slots of g rows per range, `ranges` ranges.
-WsLayout ws_layout(int g, int D, long long ranges) {
+// Caller or library workspace: split partials only (no zeroing needed).
+WsLayout ws_layout(int g, int D, long long grid) {
     WsLayout w;
     w.lse = 0;
-    w.opart = round256(sizeof(float) * 2 * ranges * g);
-    w.total = w.opart + round256(sizeof(float) * 2 * ranges * g * D);
+    w.opart = round256(sizeof(float) * 2 * grid * g);
+    w.total = w.opart + round256(sizeof(float) * 2 * grid * g * D);
     return w;
 }
 
@@ -340,7 +339,7 @@ size_t pgd_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t
     DeviceState *d = nullptr;
     if (device_state(&d) != PGD_OK) return 0;
     const long long grid = static_cast<long long>(d->sms) * kMaxCtasPerSmForSizing;
-    return ws_layout(num_q_heads / num_kv_heads, head_dim, grid * kRangesPerShare).total;
+    return ws_layout(num_q_heads / num_kv_heads, head_dim, grid).total;
 }
 
 }  // extern "C"
@@ -408,13 +407,10 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     if (grid > (1LL << 24)) return PGD_ERR_INVALID_ARG;
 
     // ---- workspace --------------------------------------------------------------
-    // a CTA's share may be cut into its main part and kTailChunks chunks
-    const WsLayout lay = ws_layout(rows, head_dim, grid * kRangesPerShare);
+    const WsLayout lay = ws_layout(rows, head_dim, grid);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // arrival counters per unit, then a claim counter per CTA and a done count
-    if ((st = ensure_counters(d, static_cast<long long>(num_seqs) * num_kv_heads + grid + 1, s)) !=
-        PGD_OK)
+    if ((st = ensure_counters(d, static_cast<long long>(num_seqs) * num_kv_heads, s)) != PGD_OK)
         return st;
     if (!ws) {
         std::lock_guard<std::mutex> lk(g_mu);
@@ -473,7 +469,6 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
     p.rows = rows;
     p.out_f32 = out_f32 ? 1 : 0;
     p.wait_ns = g_wait_ns.load();
-    p.tails_ok = 1;
     a.grid = static_cast<int>(grid);
     a.stream = s;
     cudaError_t e = var.launch(a);
@@ -805,7 +800,6 @@ extern "C" pgd_status pgd_paged_decode_attention_noalloc(
     p.window = 0;
     p.rows = g;
     p.wait_ns = g_wait_ns.load();
-    p.tails_ok = 0;   // the static array holds one range per CTA and no claim counters
     a.grid = static_cast<int>(grid);
     a.stream = s;
     e = var.launch(a);

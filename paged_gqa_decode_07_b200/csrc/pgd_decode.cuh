@@ -86,9 +86,6 @@ struct DecodeParams {
     // limit of every pipeline wait in ns (kDefaultWaitNs unless a test of
     // the timeout path shortens it)
     uint64_t wait_ns;
-    // 1: tail claiming on (the workspace holds kRangesPerShare ranges per CTA
-    // and the counters the per-share claim counters, see Ranges)
-    int32_t tails_ok;
 };
 
 constexpr int kConsumerWarps = 4;
@@ -236,49 +233,11 @@ __device__ __forceinline__ long long block_scan(long long v, long long &total, M
     return v + before;
 }
 
-// The part that holds index x when [0, U) is cut into G equal parts
-// [c*U/G, (c+1)*U/G) (all non-empty since G <= U).
+// The CTA that holds work index x (ranges are [c*U/G, (c+1)*U/G), all
+// non-empty since G <= U).
 __device__ __forceinline__ long long cta_of(long long x, long long U, long long G) {
     return ((x + 1) * G - 1) / U;
 }
-
-// Tail claiming.  CTA c's share of the work is [c*U/G, (c+1)*U/G).  SMs
-// stream at rates some 10 % apart, so with shares fixed in advance the
-// slowest CTA would set the step time.  With tails on, the last eighth of
-// every share is cut into kTailChunks chunks that any CTA may claim (one
-// atomic per claim) once it has finished its own main part: first its own
-// chunks, then those of up to kStealReach shares to its right, so a fast CTA
-// takes over the tail of a slow neighbour.  The cut is fixed: range r below
-// is the same work whoever processes it, so the split partials and their
-// merge order, and hence the bits of the result, do not depend on who claims
-// what.
-constexpr int kTailChunks = 4;
-constexpr int kRangesPerShare = kTailChunks + 1;     // main part + chunks
-constexpr int kStealReach = 8;
-
-struct Ranges {
-    long long U, G;
-    bool tails;
-    // share c: its main part is range kRangesPerShare * c, chunk i is range
-    // kRangesPerShare * c + 1 + i (work order); without tails range c is share c
-    __device__ __forceinline__ long long main_len(long long len) const {
-        return tails ? len - len / 8 : len;
-    }
-    __device__ __forceinline__ long long start(long long r) const {
-        if (!tails) return r * U / G;
-        const long long c = r / kRangesPerShare, i = r % kRangesPerShare;
-        const long long a = c * U / G, len = (c + 1) * U / G - a, m = main_len(len);
-        return i == 0 ? a : a + m + (i - 1) * (len - m) / kTailChunks;
-    }
-    __device__ __forceinline__ long long of(long long x) const {   // the range holding x
-        const long long c = cta_of(x, U, G);
-        if (!tails) return c;
-        const long long a = c * U / G, len = (c + 1) * U / G - a, m = main_len(len);
-        const long long off = x - a;
-        if (off < m) return c * kRangesPerShare;
-        return c * kRangesPerShare + 1 + cta_of(off - m, len - m, kTailChunks);
-    }
-};
 
 // Work weight of one (sequence, KV head) unit of n tiles: its tiles plus a
 // fixed cost, so that a CTA given many short units gets fewer of them.
@@ -390,8 +349,9 @@ __device__ __forceinline__ long long lds64(uint32_t a) {
 // pass, and the partial rows are read several pieces at a time so that the L2
 // round trips overlap.
 template <int D>
-__device__ __forceinline__ void merge_unit(const DecodeParams &p, long long ua, const Ranges &rg,
-                                           long long c_first, long long c_last, int s, int h) {
+__device__ __forceinline__ void merge_unit(const DecodeParams &p, long long ua, long long U,
+                                           long long G, long long c_first, long long c_last,
+                                           int s, int h) {
     constexpr int V4 = D / 4;                      // float4 columns per row
     constexpr int MAXC = (V4 + 7) / 8;             // columns per thread and pass
     const int R = p.rows, g = p.group;
@@ -401,7 +361,7 @@ __device__ __forceinline__ void merge_unit(const DecodeParams &p, long long ua, 
     // output row of query row `head`: query token head / g, head h*g + head % g
     const long long orow =
         ((long long)s * p.q_len + head / g) * p.num_q_heads + (long long)h * g + head % g;
-    auto slot_of = [&](long long c) { return 2 * c + ((ua <= rg.start(c)) ? 0 : 1); };
+    auto slot_of = [&](long long c) { return 2 * c + ((ua <= c * U / G) ? 0 : 1); };
     // One pass over the pieces in order, NG at a time with all their loads in
     // flight: running max M, weight sum W and weighted sum acc, rescaled
     // whenever M grows (the online softmax merge).
@@ -580,9 +540,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
     // CTAs beyond the work count get no range, so every range is non-empty
     const long long G = min((long long)gridDim.x, U);
     const long long u0 = cta < G ? cta * U / G : 0, u1 = cta < G ? (cta + 1) * U / G : 0;
-    // tails when every share is long enough for its chunks to be non-empty
-    const Ranges rg{U, G, p.tails_ok != 0 && U >= 64 * G};
-    const long long u1m = u0 + rg.main_len(u1 - u0);   // end of this CTA's main part
     if (U == 0) {             // every context is empty
         zero_fill(tid, kThreads, gridDim.x);
         return;
@@ -647,12 +604,11 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         // First it writes the empty units (spread over the G CTAs that have work).
         zero_fill(lane, 32, G);
         if (p.k_new == nullptr) return;
-        // (the main part only: the producer appends itself in tail chunks)
         Cursor cur = first_unit<BS>(p, misc->s0, misc->pfx0, u0, win0);
         uint32_t ait = 0;
-        for (; cur.a < u1m; next_unit<BS>(cur, p)) {
+        for (; cur.a < u1; next_unit<BS>(cur, p)) {
             const long long r0 = max(0LL, u0 - cur.a);
-            const long long r1 = min((long long)(cur.n - cur.jlo), u1m - cur.a);
+            const long long r1 = min((long long)(cur.n - cur.jlo), u1 - cur.a);
             if (r0 < r1 && cur.jlo + r1 == cur.n) {
                 const uint32_t as = ait % kAppSlots;
                 bool ok = true;
@@ -700,15 +656,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             ks_l = __ldg(p.k_scale + lane);
             vs_l = __ldg(p.v_scale + lane);
         }
-        // The range being walked, [rs, re): first this CTA's main part, then
-        // each tail chunk it claims (see Ranges).  In the main part the
-        // appender warp writes the appended rows; in a chunk the producer does.
-        long long rs = u0, re = u1m;
-        bool in_main = true;
         // the segment's blocks [j0, j1) of unit c (empty: only fixed-cost slots)
         auto seg_of = [&](const Cursor &c, int &j0, int &j1) {
-            j0 = c.jlo + (int)max(0LL, rs - c.a);
-            j1 = c.jlo + (int)min((long long)(c.n - c.jlo), re - c.a);
+            j0 = c.jlo + (int)max(0LL, u0 - c.a);
+            j1 = c.jlo + (int)min((long long)(c.n - c.jlo), u1 - c.a);
         };
         // block ids of a segment's first 32 blocks, one per lane; the next
         // unit's are loaded while this unit's tiles are issued, so the walk
@@ -726,9 +677,9 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         int pf_la = 0, la_j0 = -1;
         auto look_ahead = [&](const Cursor &from) {
             la = from;
-            while (la.a < re && la.s == from.s) next_unit<BS>(la, p);
+            while (la.a < u1 && la.s == from.s) next_unit<BS>(la, p);
             la_j0 = -1;
-            if (la.a < re) {
+            if (la.a < u1) {
                 int b0, b1;
                 seg_of(la, b0, b1);
                 pf_la = first_ids(la, b0, b1);
@@ -736,59 +687,19 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             }
         };
         int pf = 0;
-        auto enter_range = [&]() {
-            if (cur.a < re) {
-                int a0, a1;
-                seg_of(cur, a0, a1);
-                pf = first_ids(cur, a0, a1);
-                look_ahead(cur);
-            }
-        };
-        // move cur forward to the unit that holds work index x (whole
-        // sequences at a time, then heads)
-        auto seek = [&](long long x) {
-            while (cur.a + (long long)(Hkv - cur.h) * cur.w <= x) {
-                cur.a += (long long)(Hkv - 1 - cur.h) * cur.w;
-                cur.h = Hkv - 1;
-                next_unit<BS>(cur, p);
-            }
-            const long long hs = (x - cur.a) / cur.w;
-            cur.h += (int)hs;
-            cur.a += hs * cur.w;
-        };
-        // the CTA whose tail chunks are claimed next: own first, then to the right
-        long long claim_share = cta;
-        int *const claims = p.counters + (long long)B * Hkv;   // [G] claims, [gridDim.x] done
-        // the producer writes the appended row of a tail-chunk unit itself
-        auto append_row = [&](const Cursor &c) {
-            int pb = __ldg(p.block_table + (long long)c.s * p.max_blocks_per_seq + c.n - 1);
-            if (pb < 0 || pb >= p.num_blocks) {
-                if (lane == 0) raise_flag(p.flags, kFlagBlockId);
-                pb = 0;
-            }
-            const long long dst = (((long long)pb * Hkv + c.h) * BS + (c.ctx - 1) % BS) * C::ROW;
-            const long long src = ((long long)c.s * Hkv + c.h) * C::ROW;
-            constexpr int RCH = C::ROW / 16;   // 16-byte chunks per row
-            for (int k = lane; k < 2 * RCH; k += 32) {
-                const bool isk = k < RCH;
-                const int off = 16 * (isk ? k : k - RCH);
-                const uint4 v =
-                    __ldg(reinterpret_cast<const uint4 *>((isk ? p.k_new : p.v_new) + src + off));
-                *reinterpret_cast<uint4 *>((isk ? p.k_cache : p.v_cache) + dst + off) = v;
-            }
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-            __syncwarp();
-        };
-        enter_range();
-        for (;;) {                                       // ranges
-        Cursor last = cur;                               // the last unit walked
-        for (; cur.a < re && ok;) {
+        if (cur.a < u1) {
+            int a0, a1;
+            seg_of(cur, a0, a1);
+            pf = first_ids(cur, a0, a1);
+            look_ahead(cur);
+        }
+        for (; cur.a < u1 && ok;) {
             int j0, j1;                                  // absolute blocks
             seg_of(cur, j0, j1);
             Cursor nxt = cur;
             next_unit<BS>(nxt, p);
             int pf_next = 0;
-            if (nxt.a < re) {
+            if (nxt.a < u1) {
                 int b0, b1;
                 seg_of(nxt, b0, b1);
                 if (nxt.s == cur.s && b0 == j0) {
@@ -801,7 +712,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     look_ahead(nxt);
                 }
             }
-            last = cur;
             if (j0 >= j1) {          // the range holds only this unit's fixed-cost slots
                 cur = nxt;
                 pf = pf_next;
@@ -875,7 +785,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     const uint32_t slot = it % NSTAGES;
                     if (lane == 0 && it >= (uint32_t)NSTAGES)
                         ok = mbar_wait_bounded(bar_empty + 8 * slot, ((it / NSTAGES) - 1) & 1, p.wait_ns);
-                    if (app_seg && in_main && jj + nb == j1 && lane == 0 && ok) {
+                    if (app_seg && jj + nb == j1 && lane == 0 && ok) {
                         // the appended row is in this stage: wait for its write
                         const uint32_t as = ait % kAppSlots;
                         ok = mbar_wait_bounded(app_done + 8 * as, (ait / kAppSlots) & 1, p.wait_ns);
@@ -884,7 +794,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
-                    if (app_seg && !in_main && jj + nb == j1) append_row(cur);
                     const uint32_t full = bar_full + 8 * slot;
                     if (lane == 0) mbar_arrive_expect_tx(full, (uint32_t)(nb * 2 * C::TILE));
                     const uint32_t dK = sbase + slot * C::STAGE, dV = dK + C::STAGE_KV;
@@ -907,39 +816,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             }
             cur = nxt;
             pf = pf_next;
-        }
-        if (!ok || !rg.tails) break;
-        // claim the next tail chunk: this CTA's own first, then its neighbours'
-        long long chunk = -1;
-        while (claim_share < G && claim_share <= cta + kStealReach) {
-            int i = 0;
-            if (lane == 0) i = atomicAdd(claims + claim_share, 1);
-            i = __shfl_sync(0xffffffffu, i, 0);
-            if (i < kTailChunks) {
-                chunk = claim_share * kRangesPerShare + 1 + i;
-                break;
-            }
-            ++claim_share;
-        }
-        if (chunk < 0) break;
-        rs = rg.start(chunk);
-        re = rg.start(chunk + 1);
-        in_main = false;
-        cur = last;                                      // cur.a <= rs: walk forward
-        seek(rs);
-        enter_range();
-        }                                                // ranges
-        if (rg.tails && ok) {
-            // this CTA has made its last claim; the last CTA to get here resets
-            // the claim counters for the next launch (the acquire-release count
-            // orders every claim before it)
-            int prev = 0;
-            if (lane == 0) prev = atom_add_acq_rel_gpu(claims + gridDim.x, 1);
-            prev = __shfl_sync(0xffffffffu, prev, 0);
-            if (prev == (int)G - 1) {
-                for (long long c = lane; c < G; c += 32) claims[c] = 0;
-                if (lane == 0) claims[gridDim.x] = 0;
-            }
         }
         if (!ok && lane == 0) raise_flag(p.flags, kFlagTimeout);
         if (lane == 0) {
@@ -1005,10 +881,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         auto orow = [&](int r) -> long long {
             return ((long long)s * p.q_len + r / g) * p.num_q_heads + (long long)h * g + r % g;
         };
-        // partial results: slot 2r for the first segment of range r, 2r+1 for
-        // its last
-        const long long rseg = rg.of(useg);
-        const long long pslot = 2 * rseg + (useg == rg.start(rseg) ? 0 : 1);
+        // partial results: slot 2c for the CTA's first segment, 2c+1 for its last
+        const long long pslot = 2 * cta + (useg == u0 ? 0 : 1);
         constexpr int CPR = D / 8;   // 8-float chunks per row
         // (A + B) / L (two merge buffers) or A / L (one) for rows r0 .. r0 + 7,
         // 8 consecutive dims per step: the output, or this CTA's partial result
@@ -1709,14 +1583,14 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
             // unit tile range [ua, ub) in work space and the CTAs that share it
             const long long ua = useg - (j0 - jlo);
             const long long ub = ua + (nunit - jlo);
-            const long long c_first = rg.of(ua), c_last = rg.of(ub - 1);
+            const long long c_first = cta_of(ua, U, G), c_last = cta_of(ub - 1, U, G);
             if (tid == 0) {
                 const int prev = atom_add_acq_rel_gpu(p.counters + (long long)s * Hkv + h, 1);
                 misc->is_last = (prev == (int)(c_last - c_first));
             }
             named_bar_sync(kBarConsumers, kConsumers);
             if (misc->is_last) {
-                merge_unit<D>(p, ua, rg, c_first, c_last, s, h);
+                merge_unit<D>(p, ua, U, G, c_first, c_last, s, h);
                 if (tid == 0) p.counters[(long long)s * Hkv + h] = 0;
             }
         }

@@ -404,44 +404,3 @@ def test_prepared_calls_give_the_same_bits():
                            8, 128, 16, w.scale, max_context_len=w.max_context_len)
     torch.cuda.synchronize()
     assert torch.equal(out2.view(torch.int16), out3.view(torch.int16))
-
-
-# --------------------------------------------------------------------------- #
-# tail claiming: the last eighth of every CTA's share is cut into chunks that
-# any CTA may claim once it has finished its own work
-# --------------------------------------------------------------------------- #
-@pytest.mark.parametrize("num_ctas", [1, 13, 64])
-def test_tail_chunks_fixed_cut_gives_fixed_bits(num_ctas):
-    """Grids small enough that every share has tail chunks: whoever claims a
-    chunk, the cut is the same, so repeated runs give identical bits, and
-    the result matches the oracle."""
-    w = make_case([8192, 8192, 3000, 4100, 17, 1], 64, 8, 128, 16, "bf16", seed=21,
-                  name="tails")
-    d, got, ref = check_case(w, num_ctas=num_ctas)
-    outs = [d.decode(num_ctas=num_ctas)[0].clone() for _ in range(3)]
-    for o in outs:
-        assert np.array_equal(to_f64(o), got)
-
-
-def test_tail_chunks_fused_append_in_a_chunk():
-    """A unit's last block (where the appended row goes) can fall in a tail
-    chunk that another CTA claims; that CTA's producer writes the row.  The
-    cache and the output must equal the two-launch path bit for bit."""
-    from tests.gpu_helpers import dev_cache
-    w = make_case([4096, 4097, 4111, 4127, 5000, 333], 32, 8, 128, 16, "bf16", seed=22,
-                  append_last=True, name="tails-step")
-    kn, vn = _step_payload(w)
-    for nctas in (5, 29):
-        d1 = Dev(w)
-        out1 = pgd.decode_step(d1.q, dev_cache(kn), dev_cache(vn), d1.k, d1.v, d1.bt, d1.cl, 32,
-                               8, 128, 16, w.scale, max_context_len=w.max_context_len,
-                               num_ctas=nctas)
-        d2 = Dev(w)
-        d2.append()
-        out2, _ = d2.decode(num_ctas=nctas)
-        torch.cuda.synchronize()
-        ek, ev = oracle_caches(w)
-        assert np.array_equal(host_bits(d1.k), ek) and np.array_equal(host_bits(d1.v), ev)
-        assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
-        ref, _ = oracle_full(w)
-        assert_close(to_f64(out1), ref, "bf16", f"tails fused step, {nctas} CTAs")
