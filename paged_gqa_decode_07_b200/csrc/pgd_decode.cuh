@@ -329,13 +329,6 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uin
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar) : "memory");
 }
 
-// Prefetch `bytes` (a multiple of 16) at a 16-byte aligned global address
-// into L2.
-__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
-                 ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes) : "memory");
-}
-
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
     uint32_t v;
     asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
@@ -682,12 +675,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         // walk of many short units then never waits on a block-table load.
         Cursor la = cur;             // first unit of the sequence after cur's
         int pf_la = 0, la_j0 = -1;
-        // The query rows of that next sequence (all its heads, contiguous) are
-        // prefetched into L2 at the same time: under full load a segment's
-        // bulk copy of its query rows from HBM takes longer than the
-        // producer's lead over the consumers, and a stream of short units
-        // would wait on it every unit.
-        const uint32_t qseq = (uint32_t)p.q_len * p.num_q_heads * D * 2;   // bytes per sequence
         auto look_ahead = [&](const Cursor &from) {
             la = from;
             while (la.a < u1 && la.s == from.s) next_unit<BS>(la, p);
@@ -697,7 +684,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                 seg_of(la, b0, b1);
                 pf_la = first_ids(la, b0, b1);
                 la_j0 = b0;
-                if (lane == 0) bulk_prefetch_l2(p.q + (long long)la.s * (qseq / 2), qseq);
             }
         };
         int pf = 0;
