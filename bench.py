@@ -759,13 +759,20 @@ def _oracle_setup(w):
     return oracle, kc, vc
 
 
-def _oracle_unit(oracle, w, kc, vc, s, h):
+def _oracle_unit(oracle, w, kc, vc, s, h, n_tok=None):
+    """The oracle on every query row of unit (s, h); with n_tok, on the first
+    n_tok tokens of the sequence only (a bounded sample).  Returns the K/V
+    bytes of the unit that were read (once per unit, as the GPU arm counts)."""
     g = w.group
     rs = np.full(g, s, np.int32)
     rh = np.arange(h * g, h * g + g, dtype=np.int32)
-    oracle.paged_decode_rows(w.q, kc, vc, w.block_table, w.context_lens, w.num_kv_heads,
+    cl = w.context_lens
+    if n_tok is not None and n_tok < int(cl[s]):
+        cl = cl.copy()
+        cl[s] = n_tok
+    oracle.paged_decode_rows(w.q, kc, vc, w.block_table, cl, w.num_kv_heads,
                              w.scale, rs, rh, w.k_scale, w.v_scale)
-    return int(w.context_lens[s]) * w.head_dim * 2 * w.elem_bytes
+    return int(cl[s]) * w.head_dim * 2 * w.elem_bytes
 
 
 def cpu_baseline(w, seconds: float) -> dict:
@@ -795,21 +802,28 @@ def run_reference(args, rank, world):
     w = make_workload(args.workload, seed=0)
     oracle, kc, vc = _oracle_setup(w)
     units = _oracle_units(w)
-    # each step: a bounded slice of the workload (whole units), sized so the
-    # whole run stays within about two minutes
+    # each step: a bounded sample of the workload, sized so that the whole run
+    # (warm-up and timed steps) stays within about two minutes: whole units in
+    # a fixed random order, or, when one unit alone would take longer than a
+    # step's share, the first tokens of one unit
     budget = 120.0 / max(1, args.steps + args.warmup)
+    s0, h0 = units[0]
+    n_cal = int(min(int(w.context_lens[s0]), 4096))
     t = time.perf_counter()
-    _oracle_unit(oracle, w, kc, vc, *units[0])
-    per_unit = time.perf_counter() - t
-    per_step = max(1, min(len(units), int(budget / max(per_unit, 1e-6))))
+    _oracle_unit(oracle, w, kc, vc, s0, h0, n_cal)
+    per_token = (time.perf_counter() - t) / max(1, n_cal)
+    step_tokens = max(w.block_size, int(budget / max(per_token, 1e-9)))
     pos = 0
 
     def step():
         nonlocal pos
-        b = 0
-        for _ in range(per_step):
-            b += _oracle_unit(oracle, w, kc, vc, *units[pos % len(units)])
+        b, left = 0, step_tokens
+        while left > 0:
+            s_, h_ = units[pos % len(units)]
             pos += 1
+            n = min(left, int(w.context_lens[s_]))
+            b += _oracle_unit(oracle, w, kc, vc, s_, h_, n)
+            left -= n
         return b
 
     for _ in range(args.warmup):
@@ -820,8 +834,9 @@ def run_reference(args, rank, world):
     value = nbytes / dt / 1e9
     cfg = workload_desc(w)
     cfg.update({"parallelism": "host, 1 thread", "global_batch": w.num_seqs})
-    sample = (f"{per_step} (sequence, KV head) unit(s) per step, fixed random order, "
-              f"fp64 single-threaded C oracle")
+    sample = (f"{step_tokens} context tokens of whole (sequence, KV head) units per step "
+              f"(all query rows of each unit; the first tokens of a unit when it is longer), "
+              f"fixed random order, fp64 single-threaded C oracle")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
