@@ -236,7 +236,7 @@ bool supported_group(int g) { return g >= 1 && g <= 16; }
 // (the consumers convert every element), so the same time is fewer bytes.
 // The batch is cut by tiles + this many tile-equivalents per unit.
 constexpr long long kUnitOverheadBytes = 48 * 1024;
-constexpr long long kUnitOverheadBytesFp8 = 24 * 1024;
+constexpr long long kUnitOverheadBytesFp8 = 36 * 1024;
 
 int32_t unit_cost_tiles(int head_dim, int block_size, bool fp8) {
     const long long tile_kv = 2LL * block_size * head_dim * (fp8 ? 1 : 2);
@@ -245,21 +245,24 @@ int32_t unit_cost_tiles(int head_dim, int block_size, bool fp8) {
 }
 
 // Automatic grid: one wave of resident CTAs (sms x occ), fewer for small
-// batches (at least 4 stages of tiles per CTA).  With fewer (sequence, KV
-// head) units than CTAs, the grid is rounded down to a multiple of the unit
-// count when that drops at most 1/16 of it: with units of equal length every
-// CTA then holds one piece of one unit instead of the ends of two.
+// batches (at least 4 stages of work per CTA, counting each unit's fixed
+// cost, so that a batch of many short units still fills the wave).  With
+// fewer (sequence, KV head) units than CTAs, the grid is rounded down to a
+// multiple of the unit count when that drops at most 1/16 of it: with units
+// of equal length every CTA then holds one piece of one unit instead of the
+// ends of two.
 long long auto_grid(int sms, int occ, int32_t num_seqs, int32_t num_kv_heads,
-                    int32_t max_blocks_per_seq, int32_t block_size, int32_t max_context_len) {
+                    int32_t max_blocks_per_seq, int32_t block_size, int32_t max_context_len,
+                    int32_t unit_cost) {
     long long grid = static_cast<long long>(sms) * occ;
     const long long units = static_cast<long long>(num_seqs) * num_kv_heads;
     if (units > 0 && units < grid && grid % units <= grid / 16) grid -= grid % units;
     const long long cap_tokens = static_cast<long long>(max_blocks_per_seq) * block_size;
     const long long max_ctx =
         max_context_len > 0 ? std::min<long long>(max_context_len, cap_tokens) : cap_tokens;
-    const long long tiles_upper = units * ((max_ctx + block_size - 1) / block_size);
-    const long long min_tiles = 4 * (kStageTokens / block_size);   // >= 4 stages per CTA
-    return std::max(1LL, std::min(grid, (tiles_upper + min_tiles - 1) / min_tiles));
+    const long long work_upper = units * ((max_ctx + block_size - 1) / block_size + unit_cost);
+    const long long min_work = 4 * (kStageTokens / block_size);   // >= 4 stages per CTA
+    return std::max(1LL, std::min(grid, (work_upper + min_work - 1) / min_work));
 }
 
 }  // namespace
@@ -402,7 +405,7 @@ pgd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
         const int occ = var.occ();
         if (occ <= 0) return PGD_ERR_CUDA;
         grid = auto_grid(d->sms, occ, num_seqs, num_kv_heads, max_blocks_per_seq, block_size,
-                         max_context_len);
+                         max_context_len, unit_cost_tiles(head_dim, block_size, fp8));
     }
     if (grid > (1LL << 24)) return PGD_ERR_INVALID_ARG;
 
@@ -752,7 +755,7 @@ extern "C" pgd_status pgd_paged_decode_attention_noalloc(
         const int occ = var.occ();
         if (occ <= 0) return PGD_ERR_CUDA;
         grid = auto_grid(d->sms, occ, num_seqs, num_kv_heads, max_blocks_per_seq, block_size,
-                         max_context_len);
+                         max_context_len, unit_cost_tiles(head_dim, block_size, fp8));
         const long long per_cta = 8LL * g * (head_dim + 1);
         const long long fit = std::max(1LL, static_cast<long long>(avail - 512) / per_cta);
         if (grid > fit) {

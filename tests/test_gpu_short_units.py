@@ -70,9 +70,11 @@ def test_short_units_repeat_bits():
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
 
 
+@pytest.mark.parametrize("dt", ["bf16", "e4m3"])
 @pytest.mark.parametrize("L,W", [(2, 0), (2, 20), (1, 9)])
-def test_short_units_multi_token_and_window(L, W):
-    w = make_case(short_mix(150, 1130 + L + W), 16, 4, 128, 16, "bf16", seed=1131 + L,
+def test_short_units_multi_token_and_window(L, W, dt):
+    """Several query tokens and a window on short units, both KV formats."""
+    w = make_case(short_mix(150, 1130 + L + W), 16, 4, 128, 16, dt, seed=1131 + L,
                   name="short-multi")
     rng = np.random.default_rng(1132)
     qm = to_bf16_bits(rng.standard_normal((w.num_seqs, L, 16, 128), dtype=np.float32))
@@ -80,17 +82,29 @@ def test_short_units_multi_token_and_window(L, W):
     lse = torch.empty((w.num_seqs, L, 16), dtype=torch.float32, device="cuda")
     out = pgd.paged_decode_attention_ex(dev_bf16(qm), d.k, d.v, d.bt, d.cl, 16, 4, 128, 16,
                                         w.scale, window=W, max_context_len=w.max_context_len,
-                                        lse_out=lse)
+                                        k_scale=d.ks, v_scale=d.vs, lse_out=lse)
     torch.cuda.synchronize()
     ref, ref_lse = oracle.paged_decode_multi(qm, w.k_cache, w.v_cache, w.block_table,
-                                             w.context_lens, w.num_kv_heads, w.scale, window=W)
+                                             w.context_lens, w.num_kv_heads, w.scale, window=W,
+                                             k_scale=w.k_scale, v_scale=w.v_scale)
     got = to_f64(out)
     assert np.all(np.isfinite(got))
-    assert_close(got, ref, "bf16", f"short multi L={L} W={W}")
+    assert_close(got, ref, dt, f"short multi L={L} W={W}")
     gl = lse.cpu().numpy().astype(np.float64)
     live = np.isfinite(ref_lse)
     assert np.all(np.isneginf(gl[~live]))
     assert np.max(np.abs(gl[live] - ref_lse[live])) <= 1e-3
+
+
+@pytest.mark.parametrize("num_ctas", [1, 3, 37, 296, 2000])
+def test_short_unit_runs_next_to_split_ones(num_ctas):
+    """Runs of one-stage units between units that CTA ranges split, at grids
+    that cut the runs at every offset; the units of 1, 16, 17, 63 and 64
+    tokens cover a stage's partial and full 16-token sub-tiles."""
+    ctx = np.array([1, 16, 17, 63, 64, 2000, 5, 64, 33, 700, 48, 2, 64, 64, 0, 9, 3000, 31]
+                   * 6, np.int32)
+    w = make_case(ctx, 64, 8, 128, 16, "e4m3", seed=1160, name="short-runs")
+    check_case(w, num_ctas=num_ctas)
 
 
 @pytest.mark.parametrize("dt", ["bf16", "e4m3"])
