@@ -247,22 +247,23 @@ int32_t unit_cost_tiles(int head_dim, int block_size, bool fp8) {
 // Automatic grid: one wave of resident CTAs (sms x occ), fewer for small
 // batches (at least 4 stages of work per CTA, counting each unit's fixed
 // cost, so that a batch of many short units still fills the wave).  With
-// fewer (sequence, KV head) units than CTAs, the grid is rounded down to a
-// multiple of the unit count when that drops at most 1/16 of it: with units
+// fewer (sequence, KV head) units than CTAs, the grid is then rounded down to
+// a multiple of the unit count when that drops at most 1/8 of it: with units
 // of equal length every CTA then holds one piece of one unit instead of the
 // ends of two.
 long long auto_grid(int sms, int occ, int32_t num_seqs, int32_t num_kv_heads,
                     int32_t max_blocks_per_seq, int32_t block_size, int32_t max_context_len,
                     int32_t unit_cost) {
-    long long grid = static_cast<long long>(sms) * occ;
     const long long units = static_cast<long long>(num_seqs) * num_kv_heads;
-    if (units > 0 && units < grid && grid % units <= grid / 16) grid -= grid % units;
     const long long cap_tokens = static_cast<long long>(max_blocks_per_seq) * block_size;
     const long long max_ctx =
         max_context_len > 0 ? std::min<long long>(max_context_len, cap_tokens) : cap_tokens;
     const long long work_upper = units * ((max_ctx + block_size - 1) / block_size + unit_cost);
     const long long min_work = 4 * (kStageTokens / block_size);   // >= 4 stages per CTA
-    return std::max(1LL, std::min(grid, (work_upper + min_work - 1) / min_work));
+    long long grid = std::min(static_cast<long long>(sms) * occ,
+                              (work_upper + min_work - 1) / min_work);
+    if (units > 0 && units < grid && grid % units <= grid / 8) grid -= grid % units;
+    return std::max(1LL, grid);
 }
 
 }  // namespace
@@ -760,7 +761,7 @@ extern "C" pgd_status pgd_paged_decode_attention_noalloc(
         const long long fit = std::max(1LL, static_cast<long long>(avail - 512) / per_cta);
         if (grid > fit) {
             grid = fit;
-            if (units < grid && grid % units <= grid / 16) grid -= grid % units;
+            if (units < grid && grid % units <= grid / 8) grid -= grid % units;
         }
     }
     if (grid > (1LL << 24)) return PGD_ERR_INVALID_ARG;
