@@ -247,10 +247,11 @@ int32_t unit_cost_tiles(int head_dim, int block_size, bool fp8) {
 // Automatic grid: one wave of resident CTAs (sms x occ), fewer for small
 // batches (at least 4 stages of work per CTA, counting each unit's fixed
 // cost, so that a batch of many short units still fills the wave).  With
-// fewer (sequence, KV head) units than CTAs, the grid is then rounded down to
-// a multiple of the unit count when that drops at most 1/8 of it: with units
-// of equal length every CTA then holds one piece of one unit instead of the
-// ends of two.
+// fewer (sequence, KV head) units than CTAs, units of equal length should
+// split into whole pieces, one per CTA, not CTAs that hold the ends of two:
+// a small batch takes the multiple of the unit count nearest that cap, and a
+// full wave is rounded down to a multiple of it when that drops at most 1/8
+// of the wave.
 long long auto_grid(int sms, int occ, int32_t num_seqs, int32_t num_kv_heads,
                     int32_t max_blocks_per_seq, int32_t block_size, int32_t max_context_len,
                     int32_t unit_cost) {
@@ -260,9 +261,17 @@ long long auto_grid(int sms, int occ, int32_t num_seqs, int32_t num_kv_heads,
         max_context_len > 0 ? std::min<long long>(max_context_len, cap_tokens) : cap_tokens;
     const long long work_upper = units * ((max_ctx + block_size - 1) / block_size + unit_cost);
     const long long min_work = 4 * (kStageTokens / block_size);   // >= 4 stages per CTA
-    long long grid = std::min(static_cast<long long>(sms) * occ,
-                              (work_upper + min_work - 1) / min_work);
-    if (units > 0 && units < grid && grid % units <= grid / 8) grid -= grid % units;
+    const long long full = static_cast<long long>(sms) * occ;
+    const long long cap = (work_upper + min_work - 1) / min_work;
+    long long grid = std::min(full, cap);
+    if (units > 0 && units < grid) {
+        if (cap < full) {
+            const long long pieces = std::max(1LL, (cap + units / 2) / units);
+            grid = std::min(pieces, full / units) * units;
+        } else if (grid % units <= grid / 8) {
+            grid -= grid % units;
+        }
+    }
     return std::max(1LL, grid);
 }
 
