@@ -57,7 +57,7 @@ KERNEL_SOURCES = ["paged_gqa_decode_07_b200/csrc/pgd_decode.cuh",
                   "paged_gqa_decode_07_b200/csrc/pgd_ptx.cuh",
                   "paged_gqa_decode_07_b200/csrc/pgd_launch.h",
                   "paged_gqa_decode_07_b200/csrc/pgd_decode_family.cuh",
-                  "paged_gqa_decode_07_b200/csrc/pgd_api.cu"]
+                  "paged_gqa_decode_07_b200/csrc/pgd_grid.h"]
 
 
 def kernel_source_hash() -> str:

@@ -191,13 +191,9 @@ size_t pgd_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
  *                 its own zeroed device buffer (grown the same way).  Calls
  *                 that share a workspace, or run on one device at the same
  *                 time, must not overlap on the GPU.
- *   num_ctas      0 = automatic grid: one wave of resident CTAs (SM count x
- *                 CTAs per SM); with fewer (sequence, KV head) units than
- *                 that, rounded down to a multiple of the unit count when
- *                 this drops at most 1/16 of the wave; fewer for small
- *                 batches (at least four 64-token stages of tiles per CTA,
- *                 from max_context_len).  > 0 forces that many CTAs (used
- *                 to test split-count invariance)
+ *   num_ctas      0 = automatic grid (pgd_decode_grid tells which); > 0
+ *                 forces that many CTAs (used to test split-count
+ *                 invariance)
  *   stream        cudaStream_t as void*
  */
 pgd_status pgd_paged_decode_attention(
@@ -322,6 +318,27 @@ pgd_decode_math pgd_get_decode_math(void);
  */
 pgd_status pgd_debug_set_wait_limit_ns(uint64_t limit_ns);
 uint64_t pgd_debug_get_wait_limit_ns(void);
+
+/*
+ * pgd_decode_grid -- host function (no CUDA call): the CTA count of the
+ * automatic grid (num_ctas = 0) of the decode entry points on a device with
+ * `sms` multiprocessors that hold `ctas_per_sm` decode CTAs each (on a B200:
+ * 148 SMs, 2 CTAs at head_dim 128, 1 at 256).  The batch's work counts each
+ * (sequence, KV head) unit as its blocks plus a fixed cost (48 KB of K/V
+ * streaming time for bf16 caches, 36 KB for FP8), every unit taken at
+ * max_context_len (or max_blocks_per_seq * block_size when it is 0):
+ *   - grid = one wave (sms * ctas_per_sm), or fewer so that every CTA gets
+ *     at least four 64-token stages of that work (the cap);
+ *   - with fewer units than that, units of equal length should split into
+ *     whole pieces, one per CTA: a batch below the wave takes the multiple of
+ *     the unit count nearest the cap, and a full wave is rounded down to a
+ *     multiple of the unit count when that drops at most 1/8 of it.
+ * Other arguments as pgd_paged_decode_attention; fp8 = 1 for an FP8 E4M3
+ * cache.  Returns the CTA count, or 0 for invalid arguments.
+ */
+int64_t pgd_decode_grid(int32_t sms, int32_t ctas_per_sm, int32_t num_seqs,
+                        int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                        int32_t max_blocks_per_seq, int32_t max_context_len, int32_t fp8);
 
 /* ------------------------------------------------------------------------ */
 /* KV parallelism: one sequence's KV split along its length over GPUs       */

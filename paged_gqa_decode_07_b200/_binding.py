@@ -82,6 +82,8 @@ def load_library():
     lib.pgd_debug_get_wait_limit_ns.argtypes = []
     lib.pgd_kvp_plan.restype = st
     lib.pgd_kvp_plan.argtypes = [P, i32, i32, i32, i32, P, P]
+    lib.pgd_decode_grid.restype = ctypes.c_int64
+    lib.pgd_decode_grid.argtypes = [i32] * 9
     lib.pgd_decode_step.restype = st
     lib.pgd_decode_step.argtypes = [P, P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, i32, i32,
                                     f32, st, P, P, P, P, P, sz, i32, P]
@@ -387,6 +389,20 @@ def debug_set_wait_limit_ns(limit_ns: int) -> None:
 
 def debug_get_wait_limit_ns() -> int:
     return int(load_library().pgd_debug_get_wait_limit_ns())
+
+
+def decode_grid(sms: int, ctas_per_sm: int, num_seqs: int, num_kv_heads: int, head_dim: int,
+                block_size: int, max_blocks_per_seq: int, max_context_len: int = 0,
+                fp8: bool = False) -> int:
+    """CTA count of the decode entry points' automatic grid (pgd_decode_grid;
+    host only, no CUDA call).  Raises ValueError for invalid arguments."""
+    g = int(load_library().pgd_decode_grid(int(sms), int(ctas_per_sm), int(num_seqs),
+                                           int(num_kv_heads), int(head_dim), int(block_size),
+                                           int(max_blocks_per_seq), int(max_context_len),
+                                           1 if fp8 else 0))
+    if g <= 0:
+        raise ValueError("pgd_decode_grid: invalid arguments")
+    return g
 
 
 def kvp_plan(context_lens, block_size: int, world_size: int, rank: int):

@@ -13,6 +13,7 @@
 #include <vector>
 
 #include "pgd.h"
+#include "pgd_grid.h"
 #include "pgd_launch.h"
 
 namespace {
@@ -229,51 +230,6 @@ bool pick_variant(int D, int bs, int nt, bool fp8, int rows, Variant *v) {
 
 bool supported_block(int bs) { return bs == 16 || bs == 32 || bs == 64; }
 bool supported_group(int g) { return g >= 1 && g <= 16; }
-
-// Fixed cost of one (sequence, KV head) unit in a CTA (descriptor, query
-// rows, block-table fetch, first-tile latency, merge, output) expressed as the
-// K/V bytes a CTA streams in the same time.  FP8 tiles take longer per byte
-// (the consumers convert every element), so the same time is fewer bytes.
-// The batch is cut by tiles + this many tile-equivalents per unit.
-constexpr long long kUnitOverheadBytes = 48 * 1024;
-constexpr long long kUnitOverheadBytesFp8 = 36 * 1024;
-
-int32_t unit_cost_tiles(int head_dim, int block_size, bool fp8) {
-    const long long tile_kv = 2LL * block_size * head_dim * (fp8 ? 1 : 2);
-    const long long unit = fp8 ? kUnitOverheadBytesFp8 : kUnitOverheadBytes;
-    return static_cast<int32_t>((unit + tile_kv - 1) / tile_kv);
-}
-
-// Automatic grid: one wave of resident CTAs (sms x occ), fewer for small
-// batches (at least 4 stages of work per CTA, counting each unit's fixed
-// cost, so that a batch of many short units still fills the wave).  With
-// fewer (sequence, KV head) units than CTAs, units of equal length should
-// split into whole pieces, one per CTA, not CTAs that hold the ends of two:
-// a small batch takes the multiple of the unit count nearest that cap, and a
-// full wave is rounded down to a multiple of it when that drops at most 1/8
-// of the wave.
-long long auto_grid(int sms, int occ, int32_t num_seqs, int32_t num_kv_heads,
-                    int32_t max_blocks_per_seq, int32_t block_size, int32_t max_context_len,
-                    int32_t unit_cost) {
-    const long long units = static_cast<long long>(num_seqs) * num_kv_heads;
-    const long long cap_tokens = static_cast<long long>(max_blocks_per_seq) * block_size;
-    const long long max_ctx =
-        max_context_len > 0 ? std::min<long long>(max_context_len, cap_tokens) : cap_tokens;
-    const long long work_upper = units * ((max_ctx + block_size - 1) / block_size + unit_cost);
-    const long long min_work = 4 * (kStageTokens / block_size);   // >= 4 stages per CTA
-    const long long full = static_cast<long long>(sms) * occ;
-    const long long cap = (work_upper + min_work - 1) / min_work;
-    long long grid = std::min(full, cap);
-    if (units > 0 && units < grid) {
-        if (cap < full) {
-            const long long pieces = std::max(1LL, (cap + units / 2) / units);
-            grid = std::min(pieces, full / units) * units;
-        } else if (grid % units <= grid / 8) {
-            grid -= grid % units;
-        }
-    }
-    return std::max(1LL, grid);
-}
 
 }  // namespace
 
@@ -564,6 +520,17 @@ pgd_status pgd_debug_set_wait_limit_ns(uint64_t limit_ns) {
 }
 
 uint64_t pgd_debug_get_wait_limit_ns(void) { return g_wait_ns.load(); }
+
+int64_t pgd_decode_grid(int32_t sms, int32_t ctas_per_sm, int32_t num_seqs,
+                        int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                        int32_t max_blocks_per_seq, int32_t max_context_len, int32_t fp8) {
+    if (sms <= 0 || ctas_per_sm <= 0 || num_seqs < 0 || num_kv_heads <= 0 ||
+        max_blocks_per_seq <= 0 || max_context_len < 0 || (fp8 != 0 && fp8 != 1) ||
+        (head_dim != 128 && head_dim != 256) || !supported_block(block_size))
+        return 0;
+    return auto_grid(sms, ctas_per_sm, num_seqs, num_kv_heads, max_blocks_per_seq, block_size,
+                     max_context_len, unit_cost_tiles(head_dim, block_size, fp8 != 0));
+}
 
 pgd_status pgd_kvp_plan(const int32_t *context_lens, int32_t num_seqs, int32_t block_size,
                         int32_t world_size, int32_t rank, int32_t *block_start,
