@@ -5,38 +5,42 @@ namespace pgd {
 
 // Copy the K and V rows (head_dim elements of the cache type) of each (new
 // token, KV head) into physical block slot / bs, row slot % bs ("batching and
-// attention" 3.4: KV lives in fixed-size blocks).  A (token, head) pair is
-// 2 * row_vec 16-byte chunks, K's then V's; one lane moves one chunk, so a
-// warp serves one pair of 512-byte rows (bf16, head_dim 128), or two pairs of
-// 256-byte rows (FP8), or one pair in two passes (head_dim 256).  The copy is
-// bit-exact.
-__global__ void __launch_bounds__(256)
+// attention" 3.4: KV lives in fixed-size blocks).  One CTA per new token:
+// its hkv pairs of rows are 2 * row_vec 16-byte chunks each (K's then V's),
+// one thread per chunk and round.  The chunk count per pair (lg_cp) and the
+// block size (lg_bs) are powers of two, so a chunk's head, row and block are
+// shifts and masks.  The copy is bit-exact.
+constexpr int kAppendThreads = 128;
+
+__global__ void __launch_bounds__(kAppendThreads)
 kv_append_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
-                 const int64_t *__restrict__ slots, int32_t num_tokens, uint4 *k_cache,
-                 uint4 *v_cache, int32_t hkv, int32_t row_vec, int32_t bs, int64_t pool_slots,
+                 const int64_t *__restrict__ slots, uint4 *k_cache, uint4 *v_cache, int32_t hkv,
+                 int32_t row_vec, int32_t lg_cp, int32_t lg_bs, int64_t pool_slots,
                  uint32_t *flags) {
-    const int cp = 2 * row_vec;                  // chunks of one (token, head) pair
-    const int lp = cp < 32 ? cp : 32;            // lanes per pair
-    const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    const long long pair = gw * (32 / lp) + lane / lp;
-    const int sub = lane % lp;
-    if (pair >= static_cast<long long>(num_tokens) * hkv) return;
-    const int t = static_cast<int>(pair / hkv), h = static_cast<int>(pair % hkv);
+    const int t = blockIdx.x;
     const int64_t slot = __ldg(slots + t);
     if (slot < 0) return;                       // padding token
     if (slot >= pool_slots) {
-        if (sub == 0 && h == 0) raise_flag(flags, kFlagSlot);
+        if (threadIdx.x == 0) raise_flag(flags, kFlagSlot);
         return;
     }
-    const int64_t blk = slot / bs, off = slot % bs;
-    const int64_t src = (static_cast<int64_t>(t) * hkv + h) * row_vec;
-    const int64_t dst = ((blk * hkv + h) * bs + off) * row_vec;
-    for (int c = sub; c < cp; c += lp) {
+    const int64_t blk = slot >> lg_bs, off = slot & ((1 << lg_bs) - 1);
+    const int n = hkv << lg_cp;                 // chunks of the token
+    for (int i = threadIdx.x; i < n; i += kAppendThreads) {
+        const int h = i >> lg_cp, c = i & ((1 << lg_cp) - 1);
         const bool isk = c < row_vec;
         const int ch = isk ? c : c - row_vec;
-        (isk ? k_cache : v_cache)[dst + ch] = __ldg((isk ? k_new : v_new) + src + ch);
+        const int64_t src = (static_cast<int64_t>(t) * hkv + h) * row_vec + ch;
+        const int64_t dst = (((blk * hkv + h) << lg_bs) + off) * row_vec + ch;
+        (isk ? k_cache : v_cache)[dst] = __ldg((isk ? k_new : v_new) + src);
     }
+}
+
+__host__ __forceinline__ int lg2_exact(int v) {   // log2 of a power of two, else -1
+    if (v <= 0 || (v & (v - 1))) return -1;
+    int l = 0;
+    while ((1 << l) < v) ++l;
+    return l;
 }
 
 cudaError_t launch_kv_append(const void *k_new, const void *v_new, const int64_t *slots,
@@ -44,54 +48,91 @@ cudaError_t launch_kv_append(const void *k_new, const void *v_new, const int64_t
                              int32_t row_bytes, int32_t block_size, int64_t pool_slots,
                              uint32_t *flags, cudaStream_t stream) {
     const int row_vec = row_bytes / 16;
-    const int lp = 2 * row_vec < 32 ? 2 * row_vec : 32;
-    const long long pairs = static_cast<long long>(num_tokens) * hkv;
-    const long long warps = (pairs * lp + 31) / 32;
-    const long long blocks = (warps * 32 + 255) / 256;
-    kv_append_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new), slots, num_tokens,
-        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), hkv, row_vec, block_size,
-        pool_slots, flags);
+    const int lg_cp = lg2_exact(2 * row_vec), lg_bs = lg2_exact(block_size);
+    if (lg_cp < 0 || lg_bs < 0 || (static_cast<long long>(hkv) << lg_cp) > (1LL << 30))
+        return cudaErrorInvalidValue;
+    if (num_tokens == 0) return cudaSuccess;
+    kv_append_kernel<<<static_cast<unsigned>(num_tokens), kAppendThreads, 0, stream>>>(
+        static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new), slots,
+        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), hkv, row_vec, lg_cp,
+        lg_bs, pool_slots, flags);
     return cudaGetLastError();
+}
+
+// x / s rounded to nearest, the quotient IEEE division gives, for the 8
+// elements of one lane, from r = RN(1/s).  y0 = RN(x r) is within two ulps of
+// x / s.  One correction y1 = RN(y0 + (x - y0 s) r), the remainder taken in
+// one FMA, brings it within an ulp; from that faithful y1 the remainder is
+// exact and a second correction gives the correctly rounded quotient
+// (Markstein's theorem: P. Markstein, "Computation of elementary functions on
+// the IBM RISC System/6000 processor", IBM J. Res. Develop. 34(1), 1990).
+// The steps need r normal (|s| in [2^-125, 2^125]), the remainders clear of
+// underflow and the quotients clear of overflow, so with any other scale, or
+// a lane with any quotient outside [2^-100, 2^100], any |x| below 2^-100
+// (zeros and subnormals, whose signs and codes IEEE division settles) or a
+// non-finite value, the lane divides its elements with __fdiv_rn.
+__device__ __forceinline__ void div_by_scale8(float (&x)[8], float s, float r) {
+    float y[8];
+    bool fast = fabsf(s) >= 0x1p-125f && fabsf(s) <= 0x1p125f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        y[i] = x[i] * r;
+        const float ay = fabsf(y[i]), ax = fabsf(x[i]);
+        fast = fast && ay >= 0x1p-100f && ay <= 0x1p100f && ax >= 0x1p-100f;
+    }
+    if (fast) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float y1 = fmaf(fmaf(-y[i], s, x[i]), r, y[i]);
+            x[i] = fmaf(fmaf(-y1, s, x[i]), r, y1);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = __fdiv_rn(x[i], s);
+    }
 }
 
 // Quantising append: bf16 K/V rows of new tokens into an FP8 E4M3 cache
 // ("attention kernels", "what to check": FP8 KV).  Each element is divided by
-// its KV head's fp32 scale (IEEE division) and rounded to E4M3.  One warp per
-// (token, KV head); each lane turns 8 bf16 (16 bytes) into 8 bytes.
-__global__ void __launch_bounds__(256)
+// its KV head's fp32 scale (the IEEE quotient, div_by_scale8) and rounded to
+// E4M3.  One CTA per new token, as kv_append_kernel; a thread turns a chunk
+// of 8 bf16 (16 bytes) into 8 bytes.
+__global__ void __launch_bounds__(kAppendThreads)
 kv_append_quant_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
-                       const int64_t *__restrict__ slots, int32_t num_tokens, uint2 *k_cache,
-                       uint2 *v_cache, const float *__restrict__ k_scale,
-                       const float *__restrict__ v_scale, int32_t hkv, int32_t row_vec,
-                       int32_t bs, int64_t pool_slots, uint32_t *flags) {
-    const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (w >= static_cast<long long>(num_tokens) * hkv) return;
-    const int t = static_cast<int>(w / hkv), h = static_cast<int>(w % hkv);
+                       const int64_t *__restrict__ slots, uint2 *k_cache, uint2 *v_cache,
+                       const float *__restrict__ k_scale, const float *__restrict__ v_scale,
+                       int32_t hkv, int32_t row_vec, int32_t lg_cp, int32_t lg_bs,
+                       int64_t pool_slots, uint32_t *flags) {
+    const int t = blockIdx.x;
     const int64_t slot = __ldg(slots + t);
     if (slot < 0) return;
     if (slot >= pool_slots) {
-        if (lane == 0 && h == 0) raise_flag(flags, kFlagSlot);
+        if (threadIdx.x == 0) raise_flag(flags, kFlagSlot);
         return;
     }
-    const int64_t blk = slot / bs, off = slot % bs;
-    const int64_t src = (static_cast<int64_t>(t) * hkv + h) * row_vec;      // in uint4
-    const int64_t dst = ((blk * hkv + h) * bs + off) * row_vec;             // in uint2
-    const float ks = __ldg(k_scale + h), vs = __ldg(v_scale + h);
-    for (int c = lane; c < 2 * row_vec; c += 32) {
+    const int64_t blk = slot >> lg_bs, off = slot & ((1 << lg_bs) - 1);
+    const int n = hkv << lg_cp;
+    for (int i = threadIdx.x; i < n; i += kAppendThreads) {
+        const int h = i >> lg_cp, c = i & ((1 << lg_cp) - 1);
         const bool isk = c < row_vec;
         const int ch = isk ? c : c - row_vec;
-        const uint4 x = __ldg((isk ? k_new : v_new) + src + ch);
-        const float s = isk ? ks : vs;
+        const int64_t src = (static_cast<int64_t>(t) * hkv + h) * row_vec + ch;   // in uint4
+        const int64_t dst = (((blk * hkv + h) << lg_bs) + off) * row_vec + ch;    // in uint2
+        const float s = __ldg((isk ? k_scale : v_scale) + h);
+        const uint4 x = __ldg((isk ? k_new : v_new) + src);
         const uint32_t in[4] = {x.x, x.y, x.z, x.w};
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = unpack_bf16x2(in[k]);
+            v[2 * k] = f.x;
+            v[2 * k + 1] = f.y;
+        }
+        div_by_scale8(v, s, __frcp_rn(s));
         uint32_t b[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 f = unpack_bf16x2(in[i]);
-            b[i] = f32x2_to_e4m3x2(__fdiv_rn(f.x, s), __fdiv_rn(f.y, s));
-        }
-        (isk ? k_cache : v_cache)[dst + ch] = make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
+        for (int k = 0; k < 4; ++k) b[k] = f32x2_to_e4m3x2(v[2 * k], v[2 * k + 1]);
+        (isk ? k_cache : v_cache)[dst] = make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
     }
 }
 
@@ -100,12 +141,15 @@ cudaError_t launch_kv_append_quant(const void *k_new, const void *v_new, const i
                                    const float *k_scale, const float *v_scale, int32_t hkv,
                                    int32_t head_dim, int32_t block_size, int64_t pool_slots,
                                    uint32_t *flags, cudaStream_t stream) {
-    const long long warps = static_cast<long long>(num_tokens) * hkv;
-    const long long blocks = (warps * 32 + 255) / 256;
-    kv_append_quant_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new), slots, num_tokens,
+    const int row_vec = head_dim / 8;
+    const int lg_cp = lg2_exact(2 * row_vec), lg_bs = lg2_exact(block_size);
+    if (lg_cp < 0 || lg_bs < 0 || (static_cast<long long>(hkv) << lg_cp) > (1LL << 30))
+        return cudaErrorInvalidValue;
+    if (num_tokens == 0) return cudaSuccess;
+    kv_append_quant_kernel<<<static_cast<unsigned>(num_tokens), kAppendThreads, 0, stream>>>(
+        static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new), slots,
         static_cast<uint2 *>(k_cache), static_cast<uint2 *>(v_cache), k_scale, v_scale, hkv,
-        head_dim / 8, block_size, pool_slots, flags);
+        row_vec, lg_cp, lg_bs, pool_slots, flags);
     return cudaGetLastError();
 }
 
