@@ -59,32 +59,52 @@ cudaError_t launch_kv_append(const void *k_new, const void *v_new, const int64_t
     return cudaGetLastError();
 }
 
+// Two fp32 lanes in one 64-bit register for the paired FP32 instructions
+// (fma.rn.f32x2 / mul.rn.f32x2: each lane rounds as the scalar instruction).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    return static_cast<uint64_t>(__float_as_uint(lo)) |
+           (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 // x / s rounded to nearest, the quotient IEEE division gives, for the 8
-// elements of one lane, from r = RN(1/s).  y0 = RN(x r) is within two ulps of
-// x / s.  One correction y1 = RN(y0 + (x - y0 s) r), the remainder taken in
-// one FMA, brings it within an ulp; from that faithful y1 the remainder is
+// elements of one chunk, from r = RN(1/s).  y0 = RN(x r) is within two ulps
+// of x / s.  One correction y1 = RN(y0 + (x - y0 s) r), the remainder taken
+// in one FMA, brings it within an ulp; from that faithful y1 the remainder is
 // exact and a second correction gives the correctly rounded quotient
 // (Markstein's theorem: P. Markstein, "Computation of elementary functions on
 // the IBM RISC System/6000 processor", IBM J. Res. Develop. 34(1), 1990).
-// The steps need r normal (|s| in [2^-125, 2^125]), the remainders clear of
-// underflow and the quotients clear of overflow, so with any other scale, or
-// a lane with any quotient outside [2^-100, 2^100], any |x| below 2^-100
-// (zeros and subnormals, whose signs and codes IEEE division settles) or a
-// non-finite value, the lane divides its elements with __fdiv_rn.
+// The steps need r normal, the remainders clear of underflow and the
+// quotients clear of overflow: with |s| in [2^-40, 2^40] and every |x| in
+// [2^-60, 2^60] all of that holds (quotients within [2^-100, 2^100]).  Any
+// other chunk (zeros and subnormals, whose signs and codes IEEE division
+// settles, non-finite values, extreme magnitudes or scales) divides with
+// __fdiv_rn.  The steps run on pairs of elements.
 __device__ __forceinline__ void div_by_scale8(float (&x)[8], float s, float r) {
-    float y[8];
-    bool fast = fabsf(s) >= 0x1p-125f && fabsf(s) <= 0x1p125f;
+    bool fast = fabsf(s) >= 0x1p-40f && fabsf(s) <= 0x1p40f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        y[i] = x[i] * r;
-        const float ay = fabsf(y[i]), ax = fabsf(x[i]);
-        fast = fast && ay >= 0x1p-100f && ay <= 0x1p100f && ax >= 0x1p-100f;
-    }
+    for (int i = 0; i < 8; ++i) fast = fast && fabsf(x[i]) >= 0x1p-60f && fabsf(x[i]) <= 0x1p60f;
     if (fast) {
+        const uint64_t r2 = f2_pack(r, r), ns2 = f2_pack(-s, -s);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float y1 = fmaf(fmaf(-y[i], s, x[i]), r, y[i]);
-            x[i] = fmaf(fmaf(-y1, s, x[i]), r, y1);
+        for (int i = 0; i < 8; i += 2) {
+            const uint64_t xv = f2_pack(x[i], x[i + 1]);
+            const uint64_t y0 = f2_mul(xv, r2);
+            const uint64_t y1 = f2_fma(f2_fma(y0, ns2, xv), r2, y0);
+            const uint64_t q = f2_fma(f2_fma(y1, ns2, xv), r2, y1);
+            x[i] = f2_lo(q);
+            x[i + 1] = f2_hi(q);
         }
     } else {
 #pragma unroll

@@ -1,8 +1,9 @@
 """The quantising append's per-element division, bit for bit against the
 oracle (the IEEE single-precision quotient x / s, then its E4M3 code): every
 bf16 value (NaN payloads aside) divided by scales that put quotients on and
-within a few ulps of E4M3 rounding midpoints, at the ends of the range where
-the kernel falls back to IEEE division, and at random."""
+within a few ulps of E4M3 rounding midpoints, at and past the ends of the
+range where the kernel's reciprocal-and-correction path gives way to IEEE
+division, and at random."""
 import numpy as np
 import pytest
 import torch
@@ -50,6 +51,13 @@ SCALE_SETS = {
     "edges": np.array([1.0, 2.0, 0.5, 2.0 ** -125, 2.0 ** 125, 2.0 ** -126, 2.0 ** 126, 1e-40,
                        3e38, 1.5 * 2.0 ** -124, 448 / 3.0, 0.0071, 1 / 448, 7.0, 1e-20, 1e20],
                       np.float32),
+    # scales at and near the ends of the fast path's range [2^-40, 2^40], whose
+    # quotients of the largest and smallest fast-path values (2^+-60) reach
+    # 2^+-100
+    "fast_edges": np.array([2.0 ** 40, 2.0 ** -40, 2.0 ** 40 * (1 - 2.0 ** -24),
+                            2.0 ** -40 * (1 + 2.0 ** -23), 1.37 * 2.0 ** 39, 1.9 * 2.0 ** -39,
+                            1e12, 1e-12, 3.0, 5.0, 0.3, 0.7, 1.1e-7, 9.9e6, 2.0 ** 20 + 1,
+                            3 * 2.0 ** -20], np.float32),
 }
 
 
