@@ -94,7 +94,8 @@ const char *pgd_version(void);
  *   k_cache, v_cache  device, HND layout above, 16-byte aligned; rows that no
  *                  token maps to are left untouched.
  *   num_tokens >= 0 (0 enqueues nothing); head_dim in {128, 256};
- *   block_size in {16, 32, 64}; num_kv_heads >= 1.
+ *   block_size in {16, 32, 64}; num_kv_heads in 1 .. 65536 (more is
+ *   PGD_ERR_UNSUPPORTED).
  * The copy is bit-exact.  Two tokens mapped to the same slot race (the
  * result is one of them).
  */
@@ -118,7 +119,8 @@ pgd_status pgd_kv_append(const void *k_new, const void *v_new,
  *   slot_mapping      device int64 [num_tokens], as pgd_kv_append
  *   k_cache, v_cache  device E4M3 bytes, HND layout, 8-byte aligned
  *   k_scale, v_scale  device fp32 [num_kv_heads] (the scales the decode uses)
- *   head_dim in {128, 256}; block_size in {16, 32, 64}.
+ *   head_dim in {128, 256}; block_size in {16, 32, 64}; num_kv_heads in
+ *   1 .. 65536.
  * Bit-exact with that definition.
  */
 pgd_status pgd_kv_append_quant(const void *k_new, const void *v_new,

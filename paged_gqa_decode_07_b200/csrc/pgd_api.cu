@@ -42,6 +42,9 @@ DeviceState g_dev[kMaxDevices];
 
 pgd_status cuda_fail(cudaError_t) { return PGD_ERR_CUDA; }
 
+// The append kernels index a token's chunks with 32-bit integers.
+constexpr int32_t kMaxAppendHeads = 65536;
+
 pgd_status device_state(DeviceState **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PGD_ERR_CUDA;
@@ -257,6 +260,7 @@ pgd_status pgd_kv_append(const void *k_new, const void *v_new, const int64_t *sl
     if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0) return PGD_ERR_INVALID_ARG;
     if (kv_dtype != PGD_KV_BF16 && kv_dtype != PGD_KV_FP8_E4M3) return PGD_ERR_INVALID_ARG;
     if (head_dim != 128 && head_dim != 256) return PGD_ERR_UNSUPPORTED;
+    if (num_kv_heads > kMaxAppendHeads) return PGD_ERR_UNSUPPORTED;
     if (!supported_block(block_size)) return PGD_ERR_UNSUPPORTED;
     if (num_tokens == 0) return PGD_OK;
     if (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache) return PGD_ERR_INVALID_ARG;
@@ -281,6 +285,7 @@ pgd_status pgd_kv_append_quant(const void *k_new, const void *v_new, const int64
                                void *stream) {
     if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0) return PGD_ERR_INVALID_ARG;
     if (head_dim != 128 && head_dim != 256) return PGD_ERR_UNSUPPORTED;
+    if (num_kv_heads > kMaxAppendHeads) return PGD_ERR_UNSUPPORTED;
     if (!supported_block(block_size)) return PGD_ERR_UNSUPPORTED;
     if (num_tokens == 0) return PGD_OK;
     if (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache || !k_scale || !v_scale)

@@ -138,7 +138,7 @@ def test_decode_ex_host_validation(lib, q_len, window, kw, status):
 @pytest.mark.parametrize("kw,status", [
     (dict(n=-1), INVALID), (dict(D=96), UNSUPPORTED), (dict(bs=128), UNSUPPORTED),
     (dict(dt=3), INVALID), (dict(kn=None), INVALID), (dict(kn=MIS), INVALID),
-    (dict(n=0, kn=None), OK),
+    (dict(n=0, kn=None), OK), (dict(Hkv=65537), UNSUPPORTED), (dict(Hkv=65537, n=0), UNSUPPORTED),
 ])
 def test_kv_append_host_validation(lib, kw, status):
     a = dict(kn=A, vn=A, sl=A, n=4, kc=A, vc=A, Hkv=2, D=128, bs=16, nb=8, dt=0)
