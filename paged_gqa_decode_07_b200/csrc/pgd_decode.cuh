@@ -497,19 +497,22 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
     }
 
     // units with an empty context: out = 0, lse = -inf for all their query
-    // rows; thread t of nt per CTA, CTA c of nc
-    auto zero_fill = [&](int t, int nt, long long nc) {
-        for (long long v = cta + nc * t; v < (long long)B * Hkv; v += nc * nt) {
+    // rows.  Warp w of nw takes units w, w + nw, ...; its lanes write each
+    // empty unit's q_len runs of g rows in 16-byte pieces.
+    auto zero_fill = [&](long long w, long long nw) {
+        const int ln = tid & 31;
+        const int pieces = g * D * (p.out_f32 ? 4 : 2) / 16;   // of g rows
+        for (long long v = w; v < (long long)B * Hkv; v += nw) {
             const int s = (int)(v / Hkv), h = (int)(v % Hkv);
-            if (ctx_of<BS>(p, s) != 0) continue;
+            if (ctx_of<BS>(p, s) != 0) continue;   // the same length in every lane
             for (int i = 0; i < p.q_len; ++i) {
                 const long long row0 =
                     ((long long)s * p.q_len + i) * p.num_q_heads + (long long)h * g;
-                const int words = p.out_f32 ? 2 * g * D : g * D;   // 16-bit words
-                uint16_t *o = p.out + row0 * D * (p.out_f32 ? 2 : 1);
-                for (int e = 0; e < words; ++e) o[e] = 0;
+                uint4 *o = reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(p.out) +
+                                                     row0 * D * (p.out_f32 ? 4 : 2));
+                for (int c = ln; c < pieces; c += 32) o[c] = make_uint4(0u, 0u, 0u, 0u);
                 if (p.lse_out)
-                    for (int e = 0; e < g; ++e) p.lse_out[row0 + e] = -INFINITY;
+                    for (int e = ln; e < g; e += 32) p.lse_out[row0 + e] = -INFINITY;
             }
         }
     };
@@ -541,7 +544,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
     const long long G = min((long long)gridDim.x, U);
     const long long u0 = cta < G ? cta * U / G : 0, u1 = cta < G ? (cta + 1) * U / G : 0;
     if (U == 0) {             // every context is empty
-        zero_fill(tid, kThreads, gridDim.x);
+        zero_fill(cta * (kThreads / 32) + (tid >> 5), (long long)gridDim.x * (kThreads / 32));
         return;
     }
     if (u0 >= u1) return;   // nothing in flight, no barrier shared past this point
@@ -601,8 +604,9 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
         // before async-proxy reads, and signals the producer, which waits for
         // the signal before loading that block.  Only this CTA reads the
         // unit's last tile, so no other CTA can see the row half-written.
-        // First it writes the empty units (spread over the G CTAs that have work).
-        zero_fill(lane, 32, G);
+        // First it writes the empty units (one appender warp in each of the
+        // G CTAs that have work).
+        zero_fill(cta, G);
         if (p.k_new == nullptr) return;
         Cursor cur = first_unit<BS>(p, misc->s0, misc->pfx0, u0, win0);
         uint32_t ait = 0;
